@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200 — prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (`value`): chunked-prefill throughput, tokens/s over all N GPUs, on the
+H = 96, d = 128 prefill workload (B=4, T=8192, chunk 64, bf16 I/O, fp32 state).
+A step is one kda_forward_chunked call over that batch.  The same line carries the
+decode workload (B=256, H=96, 20 chained in-place steps; GB/s of state traffic) and
+the full layer workload (B=2, T=16384; tokens/s), each with its roofline.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of the
+workload (heads and sequences are independent — no data-path collective), a barrier
+brackets the timed region and the time is the max over ranks.  `value` is the
+aggregate (N x per-rank tokens) / max time: weak scaling.
+
+`--impl reference` times the fp64 CPU oracle (the only other place this file runs
+`oracle/`) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA tokens/s (prefill, H=96 d=128) and decode GB/s; fraction of roofline"
+PREFILL = "prefill_bf16_B4_T8192_H96_d128"
+DECODE = "decode_bf16_B256_H96_d128_x20"
+LAYER = "layer_bf16_B2_T16384_H96_d128"
+L2_BYTES = 126 * 1024 * 1024
+
+# Algorithmic work (per token-head, d = 128, C = 64):
+#   prefill reads q, k, v, g (4 x 256 B) and beta (2 B) and writes o (256 B): 1282 B,
+#   plus the fp32 state (64 KiB per head) read if given and written at the end.
+#   layer reads q/k/v raw (768 B), g raw (256 B), b raw (2 B), gate raw (256 B) and writes
+#   out (256 B): 1538 B, plus the final state.
+#   decode reads and writes the fp32 state (2 x 64 KiB per head) and moves 1282 B of I/O.
+#   chunked FLOPs as issued on full 64-row tiles: 10*C*d + 6*d^2 = 180224 per token-head.
+PREFILL_BYTES_PER_TOKEN_HEAD = 1282
+LAYER_BYTES_PER_TOKEN_HEAD = 1538
+FLOPS_PER_TOKEN_HEAD = 180224
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--skip", default="", help="comma list of: decode,layer,e2e,cpu")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- infra
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed regions run."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            n += 1
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def kernel_source_sha():
+    import glob
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_155_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the kernel sources
+    have not changed since it was captured; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- timing
+
+
+def timed(torch, fn, steps, warmup, stream, barrier, per_launch=True):
+    """Run fn() warmup times untimed, then `steps` times bracketed by barrier + sync.
+    Returns (total_ms, [per-launch ms]) measured with CUDA events on `stream`."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for a, b in ev:
+            if per_launch:
+                a.record(stream)
+            fn()
+            if per_launch:
+                b.record(stream)
+        t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    total = t0.elapsed_time(t1)
+    launches = [a.elapsed_time(b) for a, b in ev] if per_launch else []
+    return total, launches
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    import torch
+
+    ws, rank, local = dist_env()
+    skip = set(filter(None, args.skip.split(",")))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    from gated_delta_rule_155_b200 import build, inputs
+    if rank == 0:
+        build.build()
+    barrier()
+    from gated_delta_rule_155_b200 import kda
+
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    launches_per = {}
+    res = {}
+
+    # ------------------------------------------------------------------ prefill (headline)
+    w = inputs.WORKLOADS[PREFILL]
+    B, T, H, dk, dv = w["B"], w["T"], w["H"], w["dk"], w["dv"]
+    d = inputs.prefill_inputs(B, T, H, dk, dv, io=w["io"], seed=w["seed"])
+    host = {n: d[n].pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    dv_in = {n: host[n].to(dev) for n in host}
+    out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    sT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+
+    def prefill_step():
+        kda.kda_forward_chunked(dv_in["q"], dv_in["k"], dv_in["v"], dv_in["g"], dv_in["beta"],
+                                None, out, sT, stream=stream)
+
+    clocks = Clocks(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                    else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    clocks.start()
+    total, per = timed(torch, prefill_step, args.steps, args.warmup, stream, barrier)
+    kda.kda_check_device_error(stream)
+    ms = max_over_ranks(total / args.steps)
+    launch_ms = max_over_ranks(statistics.mean(per))
+    ntok = B * T
+    value = ws * ntok / (ms / 1e3)
+    kname = "kda_chunk_tc" if (w["io"] == "bf16" and dk == 128 and dv == 128 and tc_enabled()) \
+        else "kda_chunk_simt"
+    bytes_launch = B * T * H * PREFILL_BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
+    flops_launch = B * T * H * FLOPS_PER_TOKEN_HEAD
+    achieved = bytes_launch / (launch_ms / 1e3) / 1e9
+    traffic = traffic_for(kname)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+                "peak_source": f"{pk['source']} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
+                if pk["source"] == "measured" else "fallback 6.65 TB/s",
+                "kernel": kname, "launch_ms": round(launch_ms, 4),
+                "bytes_per_launch": bytes_launch,
+                "tensor": {"flops_per_launch": flops_launch,
+                           "achieved_tflops": round(flops_launch / (launch_ms / 1e3) / 1e12, 1),
+                           "peak_tflops": pk["bf16_tflops"],
+                           "frac": round(flops_launch / (launch_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4)}}
+    launches_per["prefill"] = 1
+
+    # e2e through the C ABI from pinned host buffers: H2D inputs, kernel, D2H output
+    e2e = None
+    if "e2e" not in skip:
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for n in host:
+                    dv_in[n].copy_(host[n], non_blocking=True)
+                prefill_step()
+                out_host.copy_(out, non_blocking=True)
+
+        ne = max(1, args.e2e_steps)
+        tot_e, _ = timed(torch, e2e_step, ne, 1, stream, barrier, per_launch=False)
+        ms_e = max_over_ranks(tot_e / ne)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        e2e = {"value": round(ws * ntok / (ms_e / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out.numel() * out.element_size(),
+               "ms_per_step": round(ms_e, 3)}
+    del dv_in, out, sT, d
+    torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------------ decode
+    if "decode" not in skip:
+        wd = inputs.WORKLOADS[DECODE]
+        Bd, Hd = wd["B"], wd["H"]
+        dd = inputs.decode_inputs(Bd, Hd, wd["dk"], wd["dv"], steps=wd["steps"], io=wd["io"],
+                                  seed=wd["seed"], s0_std=wd["s0_std"])
+        state = dd["state"].to(dev)
+        steps_in = [{n: x[n].to(dev) for n in x} for x in dd["steps"]]
+        od = torch.empty((Bd, Hd, wd["dv"]), dtype=torch.bfloat16, device=dev)
+
+        def decode_run():
+            for x in steps_in:
+                kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, od, stream=stream)
+
+        reps = max(1, args.steps // 10)
+        total_d, per_d = timed(torch, decode_run, reps, max(1, args.warmup // 3), stream, barrier,
+                               per_launch=False)
+        kda.kda_check_device_error(stream)
+        ms_d = max_over_ranks(total_d / (reps * wd["steps"]))
+        state_bytes = 2 * Bd * Hd * wd["dk"] * wd["dv"] * 4
+        io_bytes = Bd * Hd * (3 * wd["dk"] * 2 + wd["dv"] * 2 * 2 + 2)
+        gbs = (state_bytes + io_bytes) / (ms_d / 1e3) / 1e9
+        res["decode"] = {
+            "workload": "kda_decode_step B=256 H=96 dk=dv=128 bf16 I/O, fp32 state in place, 20 chained steps",
+            "value": round(ws * gbs, 1), "unit": "GB/s", "ms_per_step": round(ms_d, 4),
+            "tokens_per_s": round(ws * Bd / (ms_d / 1e3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "frac_of_8TBs": round(gbs / 8000.0, 4), "traffic": traffic_for("kda_decode"),
+                         "kernel": "kda_decode", "bytes_per_launch": state_bytes + io_bytes}}
+        launches_per["decode"] = wd["steps"] * reps
+        del state, steps_in, od, dd
+        torch.cuda.empty_cache()
+
+    # ------------------------------------------------------------------ layer
+    if "layer" not in skip:
+        wl = inputs.WORKLOADS[LAYER]
+        Bl, Tl, Hl = wl["B"], wl["T"], wl["H"]
+        L = inputs.layer_inputs(Bl, Tl, Hl, wl["dk"], wl["dv"], io=wl["io"], seed=wl["seed"],
+                                conv_std=wl["conv_std"])
+        Ld = {n: (None if L[n] is None else L[n].to(dev)) for n in L}
+        ol = torch.empty((Bl, Tl, Hl, wl["dv"]), dtype=torch.bfloat16, device=dev)
+        sl = torch.empty((Bl, Hl, wl["dk"], wl["dv"]), dtype=torch.float32, device=dev)
+        need = kda.kda_layer_workspace_size(Bl, Tl, Hl, wl["dk"], wl["dv"], torch.bfloat16)
+        wsp = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+
+        def layer_step():
+            kda.kda_layer_forward(Ld["q_raw"], Ld["k_raw"], Ld["v_raw"], Ld["conv_q"], Ld["conv_k"],
+                                  Ld["conv_v"], Ld["g_raw"], Ld["A_log"], Ld["dt_bias"], Ld["b_raw"],
+                                  Ld["o_gate_raw"], Ld["o_norm_w"], out=ol, final_state=sl,
+                                  workspace=wsp if need else None, stream=stream)
+
+        nl = max(1, args.steps // 4)
+        total_l, per_l = timed(torch, layer_step, nl, max(1, args.warmup // 2), stream, barrier)
+        kda.kda_check_device_error(stream)
+        ms_l = max_over_ranks(total_l / nl)
+        bytes_l = Bl * Tl * Hl * LAYER_BYTES_PER_TOKEN_HEAD + Bl * Hl * wl["dk"] * wl["dv"] * 4
+        gbs_l = bytes_l / (ms_l / 1e3) / 1e9
+        res["layer"] = {
+            "workload": "kda_layer_forward B=2 T=16384 H=96 dk=dv=128 bf16 (conv4+SiLU, l2norm, gate, "
+                        "beta, chunked delta rule, RMSNorm x sigmoid gate)",
+            "value": round(ws * Bl * Tl / (ms_l / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms_l, 3), "workspace_bytes": need,
+            "roofline": {"bound": "hbm", "achieved": round(gbs_l, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs_l / pk["hbm_gbs"], 4),
+                         "bytes_per_step": bytes_l}}
+        launches_per["layer"] = (3 if need else 1) * nl
+        del Ld, ol, sl, wsp, L
+        torch.cuda.empty_cache()
+
+    clk = clocks.stop()
+
+    cpu = None
+    if rank == 0 and ws == 1 and "cpu" not in skip:
+        cpu = cpu_baseline_prefill(steps=1)
+
+    gpu_launches = args.steps * launches_per["prefill"] + launches_per.get("decode", 0) + \
+        launches_per.get("layer", 0)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if kname == "kda_chunk_tc" else "f32", "data": "synthetic",
+        "config": {"workload": "kda_forward_chunked B=4 T=8192 H=96 dk=dv=128 chunk=64, bf16 q/k/v/g/beta, "
+                               "fp32 state", "B": B, "T": T, "H": H, "dk": dk, "dv": dv, "chunk": 64,
+                   "l2": "inputs (4.03 GB per step) are larger than L2 (126 MB); no flush",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+        "clocks": clk, **res,
+    }
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def tc_enabled():
+    from gated_delta_rule_155_b200 import kda
+    f = getattr(kda.library(), "kda_tc_available", None)
+    return bool(f()) if f is not None else False
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+
+def cpu_baseline_prefill(steps=1):
+    """The fp64 oracle, as it stands, on a bounded sample of the prefill workload: n heads of
+    the T = 8192 sequences (heads are independent), all host threads.  Returns the
+    cpu_baseline object; value in tokens/s of the full 96-head workload."""
+    import oracle
+    from gated_delta_rule_155_b200 import inputs
+
+    w = inputs.WORKLOADS[PREFILL]
+    cores = oracle.max_threads()
+    nh = int(min(96, max(8, 2 * cores)))
+    d = inputs.prefill_inputs(1, w["T"], nh, w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    arrs = [d[n].double().numpy() for n in ("q", "k", "v", "g", "beta")]
+    best = math.inf
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.recurrent(*arrs, None, nthreads=cores)
+        best = min(best, time.perf_counter() - t0)
+    token_heads = nh * w["T"]
+    return {"value": round(token_heads / best / w["H"], 2), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{nh} heads x T={w['T']} of the prefill workload (fp64 token recurrence, "
+                      f"{token_heads} token-heads, {best:.2f} s); tokens/s = token-heads/s / 96"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from gated_delta_rule_155_b200 import inputs
+
+    w = inputs.WORKLOADS[PREFILL]
+    cores = oracle.max_threads()
+    nh = int(min(96, max(4, cores)))
+    d = inputs.prefill_inputs(1, w["T"], nh, w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    arrs = [d[n].double().numpy() for n in ("q", "k", "v", "g", "beta")]
+    for _ in range(args.warmup):
+        oracle.recurrent(*arrs, None, nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.recurrent(*arrs, None, nthreads=cores)
+        times.append(time.perf_counter() - t0)
+    mean = statistics.mean(times)
+    token_heads = nh * w["T"]
+    value = token_heads / mean / w["H"]
+    sample = (f"{nh} heads x T={w['T']} of the prefill workload per step (fp64 token recurrence); "
+              "tokens/s = token-heads/s / 96")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "kda_forward_chunked B=4 T=8192 H=96 dk=dv=128 chunk=64, bf16 q/k/v/g/beta, "
+                               "fp32 state", "B": w["B"], "T": w["T"], "H": w["H"], "dk": 128, "dv": 128,
+                   "chunk": 64, "sample": sample},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

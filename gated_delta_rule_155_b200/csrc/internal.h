@@ -1,0 +1,63 @@
+// internal.h — host-side launcher interface between the C ABI (api.cu) and the kernels.
+// Launchers assume validated arguments; they only configure and launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kda {
+
+enum IoType { IO_F32 = 0, IO_BF16 = 1 };
+
+// Chunked prefill operands.  q, k, g, v, beta, out are in `io` dtype unless the
+// *_f32 flags say the operand is float32 (used by the layer path for its
+// internally computed gate and beta).
+struct ChunkArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *s0;  // nullable
+    void *out;
+    float *sT;        // nullable
+    int B, T, H, dk, dv;
+    IoType io;
+    bool qkv_f32, g_f32, beta_f32, out_f32;
+    int *err;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v, *g, *beta;
+    float *state;
+    void *out;
+    int B, H, dk, dv;
+    IoType io;
+};
+
+struct PrologueArgs {
+    const void *q_raw, *k_raw, *v_raw, *g_raw, *b_raw;
+    const float *conv_q, *conv_k, *conv_v, *A_log, *dt_bias;
+    float *q, *k, *v, *g, *beta;  // workspace outputs, fp32
+    int B, T, H, dk, dv;
+    IoType io;
+};
+
+struct EpilogueArgs {
+    const float *o;  // [B, T, H, dv] fp32
+    const void *z;   // o_gate_raw, io dtype
+    const float *gain;
+    float eps;
+    void *out;
+    int B, T, H, dv;
+    IoType io;
+};
+
+// CUDA-core chunked kernel: any supported dtype, dk, dv in {64, 128}.
+cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
+// tcgen05 chunked kernel: bf16 I/O, dk = dv = 128.
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
+bool chunk_tc_supported(const ChunkArgs &a);
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t s);
+cudaError_t launch_epilogue(const EpilogueArgs &a, cudaStream_t s);
+cudaError_t launch_fill_state(const float *s0, float *sT, size_t n, cudaStream_t s);
+
+}  // namespace kda

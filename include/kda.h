@@ -1,0 +1,141 @@
+/*
+ * kda.h — C ABI of libkda.so: the Kimi Delta Attention (KDA) gated delta rule on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (one head; dk x dv fp32 state S; per token t):
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ * i.e. the state is decayed per key channel by exp(g_t) (g_t <= 0), corrected by
+ * the delta rule with strength beta_t along k_t, written with k_t v_t^T and read
+ * with q_t after the write.  The query scale is 1.  Sources: the open-model-atlas
+ * page "Kimi-K3 ?inspect=blocks" (self.layers: 69 KDA layers keep a state of fixed
+ * size between calls) and maxtext PR #5548's review, item 2 (KDA tensors A_log,
+ * dt_bias, conv weights and o_norm kept in F32; exp(A_log) drives the decay).
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless a comment says otherwise; the caller owns
+ *     and allocates every buffer.  The library allocates no device memory.
+ *   - Layouts are dense and row-major (last index fastest):
+ *       q, k, g : [B, T, H, dk]      v, out : [B, T, H, dv]      beta : [B, T, H]
+ *       state   : [B, H, dk, dv] fp32
+ *   - Every tensor pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ *   - Calls are asynchronous on `stream` and never synchronise it.  KDA_OK means the
+ *     arguments were valid and the kernels were launched.  Arguments are validated
+ *     before anything is launched; on any error nothing is launched and no output
+ *     is touched.  Faults inside kernels and bounded-wait timeouts surface through
+ *     kda_check_device_error() (which synchronises the stream).
+ *   - The library never aborts, exits or prints.  It is reentrant; concurrent calls
+ *     on different streams must not share output buffers.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null required pointer, non-positive size, bad enum  */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid but not built: head dims, chunk size, dtype    */
+    KDA_ERR_MISALIGNED = 3,   /* a tensor pointer is not 16-byte aligned              */
+    KDA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, attribute, ...)  */
+    KDA_ERR_TIMEOUT = 5,      /* a kernel's bounded wait gave up (device error word)  */
+    KDA_ERR_WORKSPACE = 6     /* workspace missing or smaller than required           */
+} kda_status_t;
+
+typedef enum {
+    KDA_F32 = 0,  /* q, k, v, g, beta, out (and the layer's raw inputs) are float32  */
+    KDA_BF16 = 1  /* ... are bfloat16; the state is always float32                   */
+} kda_dtype_t;
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char *kda_status_string(kda_status_t status);
+
+/* Version of this ABI (major * 100 + minor). */
+int kda_abi_version(void);
+
+/*
+ * Chunked prefill (chunkwise-parallel form of the recurrence; results equal the
+ * token-by-token recurrence up to rounding).
+ *   q, k, g       [B, T, H, dk]   io dtype; g is the per-channel log-decay (<= 0)
+ *   v             [B, T, H, dv]   io dtype
+ *   beta          [B, T, H]       io dtype, the delta-rule strength in [0, 1]
+ *   initial_state [B, H, dk, dv]  fp32, or NULL for a zero initial state
+ *   out           [B, T, H, dv]   io dtype (written)
+ *   final_state   [B, H, dk, dv]  fp32, or NULL to skip; may equal initial_state
+ *                                 (in-place state passing)
+ *   chunk         must be 64.
+ * Supported: io KDA_F32 with dk, dv in {64, 128}; io KDA_BF16 with dk = dv = 128
+ * (tensor-core path) or dk = dv = 64.  T = 0 is valid: out is untouched and
+ * final_state receives initial_state (or zeros).
+ */
+kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, const void *g,
+                                 const void *beta, const float *initial_state, void *out,
+                                 float *final_state, int B, int T, int H, int dk, int dv,
+                                 int chunk, kda_dtype_t io, kda_stream_t stream);
+
+/*
+ * One decode step: the recurrence for a single new token per sequence, with the
+ * state updated in place (read once, written once).
+ *   q, k, g [B, H, dk] io dtype; v, out [B, H, dv] io dtype; beta [B, H] io dtype;
+ *   state [B, H, dk, dv] fp32, read and overwritten.
+ * Supported: dk, dv in {64, 128}, both dtypes.
+ */
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const void *g,
+                             const void *beta, float *state, void *out, int B, int H, int dk,
+                             int dv, kda_dtype_t io, kda_stream_t stream);
+
+/*
+ * Bytes of device workspace kda_layer_forward needs for these sizes (0 when the
+ * selected kernels need none).  *bytes is written on KDA_OK.
+ */
+kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
+                                      size_t *bytes);
+
+/*
+ * KDA layer core: prologue -> chunked gated delta rule -> epilogue.
+ *   prologue  q = l2norm(SiLU(conv_q * q_raw)), k = l2norm(SiLU(conv_k * k_raw)),
+ *             v = SiLU(conv_v * v_raw)   (depthwise causal conv, kernel 4, zero history,
+ *                                          PyTorch Conv1d tap order; l2norm eps 1e-6)
+ *             g = -exp(A_log[h]) * softplus(g_raw + dt_bias),  beta = sigmoid(b_raw)
+ *   epilogue  out = o_norm_w * cast_io(o * rsqrt(mean_dv(o^2) + norm_eps)) * sigmoid(o_gate_raw)
+ * (open-model-atlas "Kimi-K3" linear_attn_config: short_conv_kernel_size 4;
+ *  atlas.klimoza.dev KimiRMSNorm excerpt; maxtext PR #5543 sigmoid output gate.)
+ *   q_raw, k_raw  [B, T, H*dk]  io dtype      v_raw       [B, T, H*dv]  io dtype
+ *   conv_q, conv_k [H*dk, 4] fp32             conv_v      [H*dv, 4]     fp32
+ *   g_raw         [B, T, H, dk] io dtype      A_log       [H]           fp32
+ *   dt_bias       [H*dk] fp32 or NULL (zero)  b_raw       [B, T, H]     io dtype
+ *   o_gate_raw    [B, T, H, dv] io dtype      o_norm_w    [dv] fp32 or NULL (ones)
+ *   initial_state / final_state as in kda_forward_chunked.
+ *   out           [B, T, H, dv] io dtype (written)
+ *   workspace     device buffer of at least kda_layer_workspace_size() bytes, 256-byte
+ *                 aligned (may be NULL when that size is 0).
+ * Supported: dk, dv in {64, 128}, both dtypes (as kda_forward_chunked).
+ */
+kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void *v_raw,
+                               const float *conv_q, const float *conv_k, const float *conv_v,
+                               const void *g_raw, const float *A_log, const float *dt_bias,
+                               const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
+                               float norm_eps, const float *initial_state, void *out,
+                               float *final_state, void *workspace, size_t workspace_bytes,
+                               int B, int T, int H, int dk, int dv, kda_dtype_t io,
+                               kda_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the library's device error word
+ * (set by a kernel whose bounded wait gave up) and any sticky CUDA error.
+ * Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA.
+ */
+kda_status_t kda_check_device_error(kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

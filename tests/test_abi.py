@@ -1,0 +1,127 @@
+"""Host-side tests of the C ABI (no GPU needed).
+
+The library must load and export every entry point ``include/kda.h`` declares, and
+every argument error must be reported before anything is launched — so these
+calls are safe without a GPU: they pass invalid arguments (null, misaligned or
+unsupported), which the library rejects on the host.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_155_b200 import build
+
+    build.build()
+    from gated_delta_rule_155_b200 import kda
+
+    return kda.library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for s in ("kda_forward_chunked", "kda_decode_step", "kda_layer_forward", "kda_status_string",
+              "kda_layer_workspace_size", "kda_check_device_error", "kda_abi_version"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for s in declared_symbols():
+        assert hasattr(lib, s), f"libkda.so does not export {s}"
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (kda_[a-z0-9_]+)\b", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = lib.kda_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.kda_status_string(99) == b"unknown status"
+    assert lib.kda_abi_version() == 100
+
+
+P = ctypes.c_void_p
+A16 = P(0x100000)  # aligned fake address: never dereferenced (every call below fails validation)
+MIS = P(0x100008)
+
+
+def _chunked(lib, q=A16, k=A16, v=A16, g=A16, beta=A16, s0=None, out=A16, sT=None,
+             B=1, T=8, H=1, dk=64, dv=64, chunk=64, io=0):
+    return lib.kda_forward_chunked(q, k, v, g, beta, s0, out, sT, B, T, H, dk, dv, chunk, io, None)
+
+
+def test_forward_chunked_rejects_bad_arguments(lib):
+    assert _chunked(lib, q=None) == 1
+    assert _chunked(lib, out=None) == 1
+    assert _chunked(lib, B=0) == 1
+    assert _chunked(lib, H=-1) == 1
+    assert _chunked(lib, T=-1) == 1
+    assert _chunked(lib, io=7) == 1
+    assert _chunked(lib, chunk=32) == 2
+    assert _chunked(lib, dk=96) == 2
+    assert _chunked(lib, dv=256) == 2
+    assert _chunked(lib, g=MIS) == 3
+    assert _chunked(lib, s0=MIS) == 3
+    assert _chunked(lib, sT=MIS) == 3
+    assert _chunked(lib, B=1 << 20, T=1 << 20) == 2
+
+
+def test_decode_rejects_bad_arguments(lib):
+    args = [A16] * 7
+    ok = lambda **kw: lib.kda_decode_step(*[kw.get(n, a) for n, a in zip("qkvgbso", args)],
+                                          kw.get("B", 2), kw.get("H", 3), kw.get("dk", 128),
+                                          kw.get("dv", 128), kw.get("io", 1), None)
+    assert ok(s=None) == 1
+    assert ok(o=None) == 1
+    assert ok(B=0) == 1
+    assert ok(dk=32) == 2
+    assert ok(v=MIS) == 3
+
+
+def test_layer_workspace_and_argument_checks(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, ctypes.byref(n)) == 0
+    N = 2 * 16 * 3
+    assert n.value >= 4 * N * (3 * 128 + 128 + 1 + 128)
+    assert lib.kda_layer_workspace_size(2, 0, 3, 128, 128, 1, ctypes.byref(n)) == 0 and n.value == 0
+    assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, None) == 1
+    assert lib.kda_layer_workspace_size(2, 16, 3, 100, 128, 1, ctypes.byref(n)) == 2
+
+    def layer(ws=A16, ws_bytes=1 << 40, q=A16, eps=1e-6, **kw):
+        return lib.kda_layer_forward(q, A16, A16, A16, A16, A16, A16, A16, None, A16, A16, None,
+                                     ctypes.c_float(eps), None, A16, None, ws, ws_bytes,
+                                     kw.get("B", 1), kw.get("T", 16), kw.get("H", 2), 128, 128, 1, None)
+    assert layer(q=None) == 1
+    assert layer(eps=-1.0) == 1
+    assert layer(q=MIS) == 3
+    assert layer(ws=None) == 6
+    assert layer(ws_bytes=16) == 6
+    assert layer(ws=P(0x100010)) == 3  # workspace must be 256-byte aligned
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The binding raises at import when libkda.so is missing — there is no fallback."""
+    import importlib.util
+    import shutil
+    src = os.path.join(ROOT, "gated_delta_rule_155_b200", "kda.py")
+    dst = tmp_path / "kda.py"
+    shutil.copy(src, dst)
+    spec = importlib.util.spec_from_file_location("kda_nolib", dst)
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,362 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances (written here, applied to the output o and, separately, to the final state):
+  * fp32 I/O:  max|gpu - ref| / max|ref|  <= 1e-4
+  * bf16 I/O (fp32 state), the 2e-2 bound relative to the RMS of the reference:
+      final state (stored in fp32):   max|gpu - ref| <= 2e-2 rms(ref)
+      outputs (stored in bf16):       |gpu - ref| <= 2e-2 rms(ref) + 2^-8 |ref|  elementwise
+    The 2^-8 |ref| term is the bf16 output format's own rounding (round-to-nearest
+    of the exact result is within half an ulp, at most 2^-8 relative): with outputs
+    whose max/RMS ratio is ~17, rounding the exact fp64 result to bf16 alone gives
+    max|err| = 0.039 rms, so no bf16-output kernel could meet 2e-2 rms without it.
+Inputs come from the seeded generators in ``gated_delta_rule_155_b200.inputs``; the
+oracle reads the same values the GPU reads (already rounded to the I/O dtype).
+Large workloads are checked on sampled heads — heads are independent, so the
+oracle computes those heads exactly — at the full sizes and launch shape the
+benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_155_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from gated_delta_rule_155_b200 import build
+
+    build.build()
+    from gated_delta_rule_155_b200 import kda as k
+
+    return k
+
+
+def f64(t):
+    return t.detach().double().cpu().numpy()
+
+
+BF16_FORMAT_REL = 2.0 ** -8
+
+
+def err(gpu, ref, io, stored_bf16=None):
+    """Error as a fraction of the allowed bound (passes when <= 1).  `stored_bf16` says
+    whether the GPU value was stored in bf16 (outputs under bf16 I/O); the final state is
+    always fp32."""
+    gpu, ref = np.asarray(gpu, np.float64), np.asarray(ref, np.float64)
+    assert np.all(np.isfinite(gpu)), "non-finite GPU output"
+    if gpu.size == 0:
+        return 0.0
+    d = np.abs(gpu - ref)
+    if io == torch.float32:
+        return np.max(d) / max(np.max(np.abs(ref)), 1e-30) / TOL_F32
+    if stored_bf16 is None:
+        stored_bf16 = True
+    bound = TOL_BF16 * max(np.sqrt(np.mean(ref * ref)), 1e-30)
+    if stored_bf16:
+        bound = bound + BF16_FORMAT_REL * np.abs(ref)
+    return float(np.max(d / bound))
+
+
+def serr(gpu, ref, io):
+    """Error of a final state (fp32 storage) as a fraction of its bound."""
+    return err(gpu, ref, io, stored_bf16=False)
+
+
+def tol(io):
+    return 1.0
+
+
+def run_prefill(kda, d, with_final=True):
+    dev = "cuda"
+    q, k, v, g, beta = (d[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    s0 = None if d["s0"] is None else d["s0"].to(dev)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    sT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if with_final else None
+    out, sT = kda.kda_forward_chunked(q, k, v, g, beta, s0, None, sT)
+    kda.kda_check_device_error()
+    return out, sT
+
+
+def oracle_prefill(d, heads=None):
+    """Oracle on all heads, or on a list of (b, h) heads gathered into one [1, T, n, .] batch."""
+    q, k, v, g, beta = (f64(d[n]) for n in ("q", "k", "v", "g", "beta"))
+    s0 = None if d["s0"] is None else f64(d["s0"])
+    if heads is None:
+        return oracle.recurrent(q, k, v, g, beta, s0)
+    bs = [b for b, _ in heads]
+    hs = [h for _, h in heads]
+    sel = lambda a: np.ascontiguousarray(a[bs, :, hs].transpose(1, 0, *range(2, a.ndim - 1))[None])
+    s0s = None if s0 is None else np.ascontiguousarray(s0[bs, hs][None])
+    return oracle.recurrent(sel(q), sel(k), sel(v), sel(g),
+                            np.ascontiguousarray(beta[bs, :, hs].T[None]), s0s)
+
+
+def check_heads(out, sT, ref_o, ref_s, heads, io):
+    o_gpu = np.stack([f64(out[b, :, h]) for b, h in heads], axis=1)[None]
+    s_gpu = np.stack([f64(sT[b, h]) for b, h in heads], axis=0)[None]
+    eo, es = err(o_gpu, ref_o, io), serr(s_gpu, ref_s, io)
+    assert eo <= 1.0, f"output error {eo:.3e} of bound"
+    assert es <= 1.0, f"state error {es:.3e} of bound"
+    return eo, es
+
+
+# ------------------------------------------------------------------------ the workloads
+
+
+def test_recurrence_f32_workload(kda):
+    """fp32, B=1, T=256, H=2, dk=dv=64: every output and the final state."""
+    w = inputs.WORKLOADS["recurrence_f32_B1_T256_H2_d64"]
+    d = inputs.prefill_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    out, sT = run_prefill(kda, d)
+    ro, rs = oracle_prefill(d)
+    assert err(f64(out), ro, torch.float32) <= 1.0
+    assert serr(f64(sT), rs, torch.float32) <= 1.0
+
+
+def test_prefill_bf16_B1_T4096_H32(kda):
+    """bf16, nonzero fp32 initial state: every head."""
+    w = inputs.WORKLOADS["prefill_bf16_B1_T4096_H32_d128"]
+    d = inputs.prefill_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"],
+                              s0_std=w["s0_std"])
+    out, sT = run_prefill(kda, d)
+    ro, rs = oracle_prefill(d)
+    assert err(f64(out), ro, torch.bfloat16) <= 1.0
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
+def test_prefill_bf16_B4_T8192_H96_sampled_heads(kda):
+    """Full-size H=96 prefill in the benchmark's launch shape; six heads checked exactly."""
+    w = inputs.WORKLOADS["prefill_bf16_B4_T8192_H96_d128"]
+    d = inputs.prefill_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    out, sT = run_prefill(kda, d)
+    heads = [(0, 0), (1, 17), (2, 48), (3, 95), (0, 71), (3, 5)]
+    ro, rs = oracle_prefill(d, heads)
+    check_heads(out, sT, ro, rs, heads, torch.bfloat16)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(sT).all()
+
+
+# ------------------------------------------------------------------------ shapes and tails
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130])
+def test_prefill_shapes_and_ragged_tails(kda, io, dk, dv, T):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(2, T, 3, dk, dv, io=ioname, seed=1000 + T + dk + dv // 2,
+                              s0_std=0.05)
+    out, sT = run_prefill(kda, d)
+    ro, rs = oracle_prefill(d)
+    assert err(f64(out), ro, io) <= tol(io)
+    assert serr(f64(sT), rs, io) <= 1.0
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_prefill_zero_length_copies_state(kda, io):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(2, 0, 3, 128, 128, io=ioname, seed=5, s0_std=0.1)
+    out, sT = run_prefill(kda, d)
+    assert out.numel() == 0
+    torch.testing.assert_close(sT.cpu(), d["s0"], rtol=0, atol=0)
+    d["s0"] = None
+    _, sT = run_prefill(kda, d)
+    assert torch.count_nonzero(sT) == 0
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_prefill_without_initial_or_final_state(kda, io):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(1, 100, 2, 128, 128, io=ioname, seed=6)
+    out, sT = run_prefill(kda, d, with_final=False)
+    assert sT is None
+    ro, _ = oracle_prefill(d)
+    assert err(f64(out), ro, io) <= tol(io)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_state_passing_in_place_across_calls(kda, io):
+    """Two calls over [0, 100) and [100, 230) with the state updated in place equal one call."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(2, 230, 3, 128, 128, io=ioname, seed=7, s0_std=0.05)
+    dev = "cuda"
+    S = d["s0"].clone().to(dev)
+    outs = []
+    for a, b in ((0, 100), (100, 230)):
+        part = [d[n][:, a:b].contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")]
+        o, _ = kda.kda_forward_chunked(*part, S, None, S)
+        outs.append(o)
+    kda.kda_check_device_error()
+    ro, rs = oracle_prefill(d)
+    assert err(f64(torch.cat(outs, 1)), ro, io) <= tol(io)
+    assert serr(f64(S), rs, io) <= 1.0
+
+
+@pytest.mark.parametrize("gval", [-40.0, -1e-4])
+def test_extreme_gates(kda, gval):
+    """Very strong (-40 per step) and very weak (-1e-4 per step) decay on every channel."""
+    d = inputs.prefill_inputs(1, 200, 2, 128, 128, io="bf16", seed=8, s0_std=0.05)
+    d["g"] = torch.full_like(d["g"], gval)
+    out, sT = run_prefill(kda, d)
+    ro, rs = oracle_prefill(d)
+    assert err(f64(out), ro, torch.bfloat16) <= 1.0
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
+@pytest.mark.parametrize("bval", [0.0, 1.0])
+def test_beta_extremes(kda, bval):
+    d = inputs.prefill_inputs(1, 150, 2, 128, 128, io="bf16", seed=9, s0_std=0.05)
+    d["beta"] = torch.full_like(d["beta"], bval)
+    out, sT = run_prefill(kda, d)
+    ro, rs = oracle_prefill(d)
+    assert err(f64(out), ro, torch.bfloat16) <= 1.0
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
+def test_prefill_is_deterministic(kda):
+    d = inputs.prefill_inputs(2, 300, 4, 128, 128, io="bf16", seed=10, s0_std=0.02)
+    o1, s1 = run_prefill(kda, d)
+    o2, s2 = run_prefill(kda, d)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+# ------------------------------------------------------------------------ decode
+
+
+def _decode_steps(kda, dd, io_t, steps):
+    dev = "cuda"
+    S = dd["state"].clone().to(dev)
+    outs = []
+    for s in range(steps):
+        st = dd["steps"][s]
+        outs.append(kda.kda_decode_step(*(st[n].to(dev) for n in ("q", "k", "v", "g", "beta")), S))
+    kda.kda_check_device_error()
+    return outs, S
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+def test_decode_small(kda, io, dk, dv):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    dd = inputs.decode_inputs(3, 5, dk, dv, steps=4, io=ioname, seed=20 + dk + dv)
+    outs, S = _decode_steps(kda, dd, io, 4)
+    st = f64(dd["state"])
+    for s in range(4):
+        x = dd["steps"][s]
+        ro, st = oracle.decode(*(f64(x[n]) for n in ("q", "k", "v", "g", "beta")), st)
+        assert err(f64(outs[s]), ro, io) <= tol(io)
+    assert serr(f64(S), st, io) <= 1.0
+
+
+def test_decode_workload_B256_H96_20_steps_sampled_heads(kda):
+    """The full decode workload (state [256, 96, 128, 128] fp32, 20 chained steps in place);
+    the outputs of every step and the final state are checked on 48 sampled heads."""
+    w = inputs.WORKLOADS["decode_bf16_B256_H96_d128_x20"]
+    dd = inputs.decode_inputs(w["B"], w["H"], w["dk"], w["dv"], steps=w["steps"], io=w["io"],
+                              seed=w["seed"], s0_std=w["s0_std"])
+    rng = np.random.default_rng(0)
+    bs = rng.integers(0, w["B"], 48)
+    hs = rng.integers(0, w["H"], 48)
+    st = f64(dd["state"][bs, hs])[None]                     # [1, 48, dk, dv]
+    outs, S = _decode_steps(kda, dd, torch.bfloat16, w["steps"])
+    for s in range(w["steps"]):
+        x = dd["steps"][s]
+        args = [f64(x[n][bs, hs])[None] for n in ("q", "k", "v", "g", "beta")]
+        ro, st = oracle.decode(*args, st)
+        assert err(f64(outs[s][bs, hs])[None], ro, torch.bfloat16) <= 1.0
+    assert serr(f64(S[bs, hs])[None], st, torch.bfloat16) <= 1.0
+
+
+def test_decode_chain_equals_prefill(kda):
+    """20 decode steps equal one prefill over the same 20 tokens (T = 1 prefill == decode)."""
+    d = inputs.prefill_inputs(2, 20, 3, 128, 128, io="f32", seed=30, s0_std=0.05)
+    dev = "cuda"
+    o_p, s_p = run_prefill(kda, d)
+    S = d["s0"].clone().to(dev)
+    for t in range(20):
+        o = kda.kda_decode_step(*(d[n][:, t].contiguous().to(dev) for n in ("q", "k", "v", "g", "beta")), S)
+        torch.testing.assert_close(o, o_p[:, t], rtol=1e-4, atol=1e-5)
+    torch.testing.assert_close(S, s_p, rtol=1e-4, atol=1e-5)
+
+
+# ------------------------------------------------------------------------ layer
+
+
+def run_layer(kda, d, with_final=True):
+    dev = "cuda"
+    to = lambda x: None if x is None else x.to(dev)
+    B, T, H, dk = d["g_raw"].shape
+    dv = d["o_gate_raw"].shape[-1]
+    sT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if with_final else None
+    out, sT = kda.kda_layer_forward(
+        to(d["q_raw"]), to(d["k_raw"]), to(d["v_raw"]), to(d["conv_q"]), to(d["conv_k"]),
+        to(d["conv_v"]), to(d["g_raw"]), to(d["A_log"]), to(d["dt_bias"]), to(d["b_raw"]),
+        to(d["o_gate_raw"]), to(d["o_norm_w"]), initial_state=to(d["s0"]), final_state=sT)
+    kda.kda_check_device_error()
+    return out, sT
+
+
+def oracle_layer(d, io, heads=None):
+    a = {n: (None if d[n] is None else f64(d[n])) for n in d}
+    io_bf16 = io == torch.bfloat16
+    if heads is None:
+        return oracle.layer(a["q_raw"], a["k_raw"], a["v_raw"], a["conv_q"], a["conv_k"], a["conv_v"],
+                            a["g_raw"], a["A_log"], a["dt_bias"], a["b_raw"], a["o_gate_raw"],
+                            a["o_norm_w"], io_bf16=io_bf16, s0=a["s0"])
+    B, T, H, dk = a["g_raw"].shape
+    dv = a["o_gate_raw"].shape[-1]
+    outs, states = [], []
+    for b, h in heads:
+        ck = slice(h * dk, (h + 1) * dk)
+        cv = slice(h * dv, (h + 1) * dv)
+        o, s = oracle.layer(a["q_raw"][b:b + 1, :, ck], a["k_raw"][b:b + 1, :, ck],
+                            a["v_raw"][b:b + 1, :, cv], a["conv_q"][ck], a["conv_k"][ck],
+                            a["conv_v"][cv], a["g_raw"][b:b + 1, :, h:h + 1], a["A_log"][h:h + 1],
+                            None if a["dt_bias"] is None else a["dt_bias"][ck], a["b_raw"][b:b + 1, :, h:h + 1],
+                            a["o_gate_raw"][b:b + 1, :, h:h + 1], a["o_norm_w"], io_bf16=io_bf16,
+                            s0=None if a["s0"] is None else a["s0"][b:b + 1, h:h + 1])
+        outs.append(o[0, :, 0])
+        states.append(s[0, 0])
+    return np.stack(outs, 1)[None], np.stack(states, 0)[None]
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d_", [64, 128])
+@pytest.mark.parametrize("T", [1, 5, 64, 150])
+def test_layer_small(kda, io, d_, T):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.layer_inputs(2, T, 3, d_, d_, io=ioname, seed=40 + T + d_, s0_std=0.05,
+                            dt_bias_std=0.5, gain_std=0.2)
+    out, sT = run_layer(kda, d)
+    ro, rs = oracle_layer(d, io)
+    assert err(f64(out), ro, io) <= tol(io)
+    assert serr(f64(sT), rs, io) <= 1.0
+
+
+def test_layer_workload_B2_T16384_H96_sampled_heads(kda):
+    """The full layer workload (bf16, unit gain, zero state) in the benchmark's launch shape."""
+    w = inputs.WORKLOADS["layer_bf16_B2_T16384_H96_d128"]
+    d = inputs.layer_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"],
+                            conv_std=w["conv_std"])
+    out, sT = run_layer(kda, d)
+    heads = [(0, 0), (1, 95), (0, 50), (1, 13)]
+    ro, rs = oracle_layer(d, torch.bfloat16, heads)
+    check_heads(out, sT, ro, rs, heads, torch.bfloat16)
+
+
+def test_layer_zero_gate_input_halves_output(kda):
+    """o_gate_raw = 0: the output is exactly half the gain-scaled normalised output of the
+    same call with a saturated gate (sigmoid(0) = 1/2)."""
+    d = inputs.layer_inputs(1, 70, 2, 128, 128, io="f32", seed=50)
+    d["o_gate_raw"] = torch.zeros_like(d["o_gate_raw"])
+    half, _ = run_layer(kda, d)
+    d["o_gate_raw"] = torch.full_like(d["o_gate_raw"], 100.0)
+    full, _ = run_layer(kda, d)
+    torch.testing.assert_close(2 * half, full, rtol=1e-6, atol=1e-6)
