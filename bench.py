@@ -66,10 +66,9 @@ def parse():
 
 
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from gated_delta_rule_155_b200.dist_util import env
+
+    return env()
 
 
 def peaks():
@@ -207,12 +206,11 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
+    from gated_delta_rule_155_b200.dist_util import aggregate_rate
+    from gated_delta_rule_155_b200.dist_util import max_over_ranks as _mor
+
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return _mor(x, dist, dev)
 
     from gated_delta_rule_155_b200 import build, inputs
     if rank == 0:
@@ -246,9 +244,8 @@ def run_ours(args):
     ms = max_over_ranks(total / args.steps)
     launch_ms = max_over_ranks(statistics.mean(per))
     ntok = B * T
-    value = ws * ntok / (ms / 1e3)
-    kname = "kda_chunk_tc" if (w["io"] == "bf16" and dk == 128 and dv == 128 and tc_enabled()) \
-        else "kda_chunk_simt"
+    value = aggregate_rate(ntok, ms, ws)
+    kname = "kda_chunk_tc" if (w["io"] == "bf16" and dk == 128 and dv == 128) else "kda_chunk_simt"
     bytes_launch = B * T * H * PREFILL_BYTES_PER_TOKEN_HEAD + B * H * dk * dv * 4
     flops_launch = B * T * H * FLOPS_PER_TOKEN_HEAD
     achieved = bytes_launch / (launch_ms / 1e3) / 1e9
@@ -382,12 +379,6 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
-
-
-def tc_enabled():
-    from gated_delta_rule_155_b200 import kda
-    f = getattr(kda.library(), "kda_tc_available", None)
-    return bool(f()) if f is not None else False
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)

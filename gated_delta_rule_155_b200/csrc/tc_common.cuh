@@ -177,6 +177,28 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
            | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor for kind::tf32 (fp32 operands read at tf32 precision), fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn, bool b_mn, bool neg_a = false)
+{
+    return (1u << 4)                        // D format: f32
+           | (2u << 7)                      // A format: tf32
+           | (2u << 10)                     // B format: tf32
+           | ((neg_a ? 1u : 0u) << 13)
+           | ((a_mn ? 1u : 0u) << 15)
+           | ((b_mn ? 1u : 0u) << 16)
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc], kind::tf32 (A: M lanes x K fp32 columns)
+KDA_DEVICE void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc));
+}
+
 // D[tmem] (+)= A[smem desc] x B[smem desc]
 KDA_DEVICE void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc)
 {

@@ -1,0 +1,61 @@
+"""Run one KDA entry point a few times on a chosen size — a driver for profilers.
+
+    python -m gated_delta_rule_155_b200.profile_case prefill --B 2 --T 4096 --H 96 --launches 3
+    python -m gated_delta_rule_155_b200.profile_case decode  --B 64 --H 96 --launches 3
+    python -m gated_delta_rule_155_b200.profile_case layer   --B 1 --T 4096 --H 96 --launches 2
+
+Inputs come from the seeded generators; nothing is checked or timed here (use the
+tests for parity and bench.py for timing).  Sizes should keep the inputs larger than
+L2 (126 MB) so DRAM counters mean something, but small enough for a profiler's
+per-kernel replay.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kind", choices=["prefill", "decode", "layer"])
+    ap.add_argument("--B", type=int, default=2)
+    ap.add_argument("--T", type=int, default=4096)
+    ap.add_argument("--H", type=int, default=96)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--launches", type=int, default=3)
+    a = ap.parse_args(argv)
+
+    from gated_delta_rule_155_b200 import build, inputs
+    build.build()
+    from gated_delta_rule_155_b200 import kda
+
+    dev = torch.device("cuda", 0)
+    if a.kind == "prefill":
+        d = inputs.prefill_inputs(a.B, a.T, a.H, a.d, a.d, io="bf16", seed=2)
+        args = [d[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+        out = torch.empty_like(args[2])
+        sT = torch.empty((a.B, a.H, a.d, a.d), device=dev)
+        for _ in range(a.launches):
+            kda.kda_forward_chunked(*args, None, out, sT)
+    elif a.kind == "decode":
+        dd = inputs.decode_inputs(a.B, a.H, a.d, a.d, steps=1, seed=3)
+        st = dd["state"].to(dev)
+        x = {n: dd["steps"][0][n].to(dev) for n in ("q", "k", "v", "g", "beta")}
+        for _ in range(a.launches):
+            kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    else:
+        L = inputs.layer_inputs(a.B, a.T, a.H, a.d, a.d, io="bf16", seed=4)
+        to = lambda t: None if t is None else t.to(dev)
+        args = [to(L[n]) for n in ("q_raw", "k_raw", "v_raw", "conv_q", "conv_k", "conv_v", "g_raw",
+                                   "A_log", "dt_bias", "b_raw", "o_gate_raw", "o_norm_w")]
+        sT = torch.empty((a.B, a.H, a.d, a.d), device=dev)
+        for _ in range(a.launches):
+            kda.kda_layer_forward(*args, final_state=sT)
+    kda.kda_check_device_error()
+    torch.cuda.synchronize()
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
