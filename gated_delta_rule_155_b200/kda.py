@@ -48,6 +48,8 @@ def _load():
     lib.kda_layer_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
     lib.kda_layer_forward.restype = i
     lib.kda_layer_forward.argtypes = [vp] * 12 + [f] + [vp] * 4 + [sz] + [i] * 5 + [i, vp]
+    lib.kda_layer_forward_noalloc.restype = i
+    lib.kda_layer_forward_noalloc.argtypes = [vp] * 12 + [f] + [vp] * 3 + [i] * 5 + [i, vp]
     lib.kda_check_device_error.restype = i
     lib.kda_check_device_error.argtypes = [vp]
     return lib
@@ -57,7 +59,9 @@ _lib = _load()
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_abi_version", "kda_forward_chunked",
                     "kda_decode_step", "kda_layer_workspace_size", "kda_layer_forward",
-                    "kda_check_device_error")
+                    "kda_layer_forward_noalloc", "kda_check_device_error")
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 
 
 def library():
@@ -181,6 +185,38 @@ def kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log,
         _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
         float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(workspace),
         ws_bytes, B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward")
+    return out, final_state
+
+
+def kda_layer_forward_noalloc(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,
+                              b_raw, o_gate_raw, o_norm_w=None, *, norm_eps=1e-6, initial_state=None,
+                              out=None, final_state=None, stream=None):
+    """kda_layer_forward with its scratch in the library's own fixed device buffer (no
+    workspace argument, no allocation inside the call except ``out`` when it is not given —
+    pass ``out`` to allocate nothing at all).  Sizes needing more than NOALLOC_SCRATCH_BYTES
+    of scratch raise KdaError (KDA_ERR_WORKSPACE).  Returns (out, final_state)."""
+    B, T, H, dk = g_raw.shape
+    dv = o_gate_raw.shape[-1]
+    io = g_raw.dtype
+    f32 = torch.float32
+    for t, s, d, n in ((q_raw, (B, T, H * dk), io, "q_raw"), (k_raw, (B, T, H * dk), io, "k_raw"),
+                       (v_raw, (B, T, H * dv), io, "v_raw"), (b_raw, (B, T, H), io, "b_raw"),
+                       (o_gate_raw, (B, T, H, dv), io, "o_gate_raw"),
+                       (conv_q, (H * dk, 4), f32, "conv_q"), (conv_k, (H * dk, 4), f32, "conv_k"),
+                       (conv_v, (H * dv, 4), f32, "conv_v"), (A_log, (H,), f32, "A_log")):
+        _need(t, s, d, n)
+    _need(dt_bias, (H * dk,), f32, "dt_bias", allow_none=True)
+    _need(o_norm_w, (dv,), f32, "o_norm_w", allow_none=True)
+    _need(initial_state, (B, H, dk, dv), f32, "initial_state", allow_none=True)
+    _need(final_state, (B, H, dk, dv), f32, "final_state", allow_none=True)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=io, device=g_raw.device)
+    _need(out, (B, T, H, dv), io, "out")
+    _check(_lib.kda_layer_forward_noalloc(
+        _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
+        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
+        float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state),
+        B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward_noalloc")
     return out, final_state
 
 

@@ -127,6 +127,36 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
                                int B, int T, int H, int dk, int dv, kda_dtype_t io,
                                kda_stream_t stream);
 
+/* Size in bytes of the built-in scratch that kda_layer_forward_noalloc uses (64 MiB). */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * kda_layer_forward_noalloc — kda_layer_forward for callers that cannot allocate device
+ * memory on their call path: a serving loop whose device memory is planned once at
+ * start-up, a plugin or callback interface that provides no allocator, or code that
+ * cannot pay for cudaMalloc (which may synchronise the device).  The paper has no
+ * counterpart to this entry point; it exists for those callers only.
+ *   Arguments, layouts and results are those of kda_layer_forward without the workspace
+ *   pair.  The caller still owns and passes every input and output.
+ *   Scratch: a library-owned device array of KDA_NOALLOC_SCRATCH_BYTES, held by every GPU
+ *   that loads the library until the process exits.  Sizes whose workspace
+ *   (kda_layer_workspace_size) exceeds it are rejected with KDA_ERR_WORKSPACE before
+ *   anything runs.  All calls share the array and it keeps the last call's contents;
+ *   each call writes every scratch byte it reads, so nothing needs clearing.  Calls that
+ *   overlap on the GPU (other streams or host threads) race on it and must be serialised
+ *   by the caller.
+ *   The first call on each device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture begins.
+ */
+kda_status_t kda_layer_forward_noalloc(const void *q_raw, const void *k_raw, const void *v_raw,
+                                       const float *conv_q, const float *conv_k,
+                                       const float *conv_v, const void *g_raw, const float *A_log,
+                                       const float *dt_bias, const void *b_raw,
+                                       const void *o_gate_raw, const float *o_norm_w,
+                                       float norm_eps, const float *initial_state, void *out,
+                                       float *final_state, int B, int T, int H, int dk, int dv,
+                                       kda_dtype_t io, kda_stream_t stream);
+
 /*
  * Synchronises `stream`, then reports and clears the library's device error word
  * (set by a kernel whose bounded wait gave up) and any sticky CUDA error.

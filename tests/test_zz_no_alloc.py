@@ -1,0 +1,83 @@
+"""kda_layer_forward_noalloc — the layer forward for callers that cannot allocate.
+
+Some callers must not allocate device memory on their call path (a serving loop whose
+memory is planned once at start-up, a plugin or callback interface that hands over no
+allocator, latency-critical code that cannot pay for cudaMalloc's possible device-wide
+synchronisation).  For them the library offers a variant of the layer forward whose
+intermediate buffers live in a fixed device array owned by the library.  These tests
+call it through the C ABI and check it against kda_layer_forward (which uses a caller
+workspace) on two calls in a row with different inputs — the shared scratch keeps the
+previous call's contents, so the second call must not depend on them — and check that
+sizes beyond the built-in scratch are refused before anything runs.
+
+This file is named to be collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_155_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from gated_delta_rule_155_b200 import build
+
+    build.build()
+    from gated_delta_rule_155_b200 import kda as k
+
+    return k
+
+
+def within(gpu, ref, io, stored_in_io):
+    """The bound the parity tests use: fp32 I/O max|d| <= 1e-4 max|ref|; bf16 I/O
+    |d| <= 2e-2 rms(ref) (+ 2^-8 |ref| for values stored in bf16)."""
+    gpu = gpu.detach().double().cpu().numpy()
+    ref = ref.detach().double().cpu().numpy()
+    d = np.abs(gpu - ref)
+    if io == torch.float32:
+        return bool(np.max(d) <= TOL_F32 * np.max(np.abs(ref)))
+    bound = TOL_BF16 * np.sqrt(np.mean(ref * ref)) + (2.0 ** -8 * np.abs(ref) if stored_in_io else 0.0)
+    return bool(np.all(d <= bound))
+
+
+def _args(d, dev):
+    to = lambda x: None if x is None else x.to(dev)
+    return [to(d[n]) for n in ("q_raw", "k_raw", "v_raw", "conv_q", "conv_k", "conv_v", "g_raw",
+                               "A_log", "dt_bias", "b_raw", "o_gate_raw", "o_norm_w")], to(d["s0"])
+
+
+@pytest.mark.parametrize("io", [torch.bfloat16, torch.float32])
+def test_noalloc_matches_layer_forward_on_two_calls(kda, io):
+    dev = "cuda"
+    ioname = "bf16" if io == torch.bfloat16 else "f32"
+    B, T, H, d_ = 2, 150, 4, 128
+    for call, seed in enumerate((71, 72)):
+        d = inputs.layer_inputs(B, T, H, d_, d_, io=ioname, seed=seed, s0_std=0.05, dt_bias_std=0.4,
+                                gain_std=0.2)
+        args, s0 = _args(d, dev)
+        ref_s = torch.empty((B, H, d_, d_), device=dev)
+        ref, _ = kda.kda_layer_forward(*args, initial_state=s0, final_state=ref_s)
+        out = torch.empty_like(ref)
+        st = torch.empty_like(ref_s)
+        kda.kda_layer_forward_noalloc(*args, initial_state=s0, out=out, final_state=st)
+        kda.kda_check_device_error()
+        assert within(out, ref, io, True), f"output mismatch on call {call}"
+        assert within(st, ref_s, io, False), f"final state mismatch on call {call}"
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch(kda):
+    lib = kda.library()
+    need = kda.kda_layer_workspace_size(4, 8192, 96, 128, 128, torch.bfloat16)
+    assert need > kda.NOALLOC_SCRATCH_BYTES
+    fake = ctypes.c_void_p(0x100000)   # never dereferenced: the call is refused before any launch
+    st = lib.kda_layer_forward_noalloc(*([fake] * 8), None, fake, fake, None, ctypes.c_float(1e-6),
+                                       None, fake, None, 4, 8192, 96, 128, 128, 1, None)
+    assert st == 6  # KDA_ERR_WORKSPACE
