@@ -26,13 +26,14 @@
 //     CV_I[j] = k_j exp(m_I - G_j)   for every j in blocks 0..I,
 // so every pair (i in block I, j <= i) gets exactly exp(G_i - G_j).  Off-diagonal
 // factors are products of in-block decays (all <= 1); only the diagonal block carries
-// factors up to exp(range_I / 2).  A channel whose decay over block I exceeds e^170
+// factors up to exp(range_I / 2).  A channel whose decay over block I exceeds e^168
 // ("bad") falls back to the block-start reference for its rows, is left out of
 // block I's diagonal in the MMA, and has that diagonal added exactly on CUDA cores.
 //
 // Precision.  bf16 operands alone would put errors of the order of one bf16 rounding
 // on top of the output's own bf16 rounding.  So the diagonal P[i][i] = q_i . k_i is
-// formed exactly in fp32 from the raw inputs, U and P enter their products as
+// formed exactly in fp32 from the raw inputs, the diagonal 16x16 blocks of the Gram get a
+// second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U and P enter their products as
 // hi + lo bf16 pairs (O += U_hi P_hi + U_lo P_hi + U_hi P_lo, S += K~^T (U_hi + U_lo)),
 // and the state is read at tf32 precision from its fp32 copy (Q^ and W kept in fp32).
 #include <cuda.h>
@@ -51,7 +52,7 @@ using namespace tc;
 constexpr int NT = 256;       // threads
 constexpr int CK = 64;        // chunk
 constexpr int DD = 128;       // dk = dv
-constexpr float BAD_LOG = -170.0f;  // block log-decays below this take the exact fallback
+constexpr float BAD_LOG = -168.0f;  // block log-decays below this take the exact fallback
 
 // shared memory layout (offsets from a 1024-byte aligned base)
 constexpr int REG_BYTES = 73728;                 // 72 KB: stage (q,k,v,g) or Gram operands
@@ -92,9 +93,12 @@ constexpr uint32_t TM_W = 128;
 constexpr uint32_t TM_UL = 192;  // bf16 (U - U_hi)^T (A operand), 32 cols, inside the Gram area
 constexpr uint32_t TM_U = 288;   // U^T, 64 cols
 constexpr uint32_t TM_O = 352;   // O^T, 64 cols
+constexpr uint32_t TM_CORR = 416;  // diagonal-block Gram correction R_lo CVd + R CVd_lo, 64 cols
 constexpr uint32_t TM_UB = 480;  // bf16 U^T (A operand), 32 cols
 
-__host__ __device__ constexpr int cv_start(int I) { return I == 0 ? 0 : I == 1 ? 16 : I == 2 ? 48 : 96; }
+// Gram column buffer: rows 0..63 are the diagonal-block columns (row j for token j);
+// rows cv_off(I) + j (j < 16 I) are block I's columns for earlier tokens.
+__host__ __device__ constexpr int cv_off(int I) { return I == 1 ? 64 : I == 2 ? 80 : 112; }
 
 struct TcParams {
     const __nv_bfloat16 *q, *k, *g, *beta;
@@ -119,7 +123,7 @@ KDA_DEVICE uint4 pack8(const float (&f)[8])
 __global__ void __launch_bounds__(NT, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                    TcParams p)
+                    const __grid_constant__ CUtensorMap tm_o, TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -152,6 +156,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int i = 0; i < 4; ++i) badcnt[i] = 0;
         fence_mbar_init();
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_g);
+        prefetch_tmap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(tslot, 512);
@@ -199,6 +204,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     };
 
     const uint32_t id_gram = idesc_bf16(128, CV_ROWS, false, false);
+    const uint32_t id_corr = idesc_bf16(128, 64, false, false);
     const uint32_t id_o0 = idesc_tf32(128, 64, false, false);
     const uint32_t id_wt = idesc_bf16(128, 64, true, false);
     const uint32_t id_u = idesc_tf32(128, 64, false, false, true);
@@ -212,6 +218,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int t0 = n * CK;
         const int nt = min(CK, T - t0);
 
+        // the previous chunk's O tile must have left X2 before this chunk writes there (after
+        // the barrier inside prep)
+        if (tid == 0) bulk_wait_read_all();
         if (!mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err)) break;
 
         // ============================================================ prep
@@ -220,71 +229,43 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int cb = warp >> 2;         // channel block (64 channels)
         const int qq = lane & 3;          // token quarter inside the block
         const int a = lane >> 2;          // 16-byte chunk (8 channels) inside the channel block
-        // per (token s of this lane's quarter, channel e of its 8):
-        //   e1 = exp(G_i - G_blockstart) (prefix product, <= 1), e2 = exp(G_blockend - G_i) (<= 1),
-        //   Gl = G_i - G_blockstart (log), Lb = block log-decay
-        float e1[4][8], e2[4][8], Gl[4][8], Lb[8];
+        // per (token s of this lane's quarter, channel e of its 8), with SC = 2^120:
+        //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
+        //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
+        // formed from log-domain prefix sums (no partial product can underflow); both are
+        // normal numbers for block log-decays down to -168 (SC e^-168 ~ e^-84.8), so the
+        // midpoint factors below are per-channel constants times E1 or E2.
+        constexpr float INV_SC = 7.523164e-37f;    // 2^-120
+        constexpr float LN_SC = 83.17766f;         // 120 ln 2
+        float E1[4][8], E2[4][8], Lb[8];
         {
-            float al[4][8];
+            float gl[4][8];
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const int i = 16 * B + 4 * qq + s;
                 float gf[8];
                 unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), gf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    al[s][e] = __expf(gf[e]);
-                    Gl[s][e] = (s == 0 ? 0.0f : Gl[s - 1][e]) + gf[e];
-                }
+                for (int e = 0; e < 8; ++e) gl[s][e] = (s == 0 ? 0.0f : gl[s - 1][e]) + gf[e];
             }
-            float tot[8], excl[8], sexc[8], lexc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                e1[0][e] = al[0][e];
-                e1[1][e] = e1[0][e] * al[1][e];
-                e1[2][e] = e1[1][e] * al[2][e];
-                e1[3][e] = e1[2][e] * al[3][e];
-                e2[3][e] = 1.0f;
-                e2[2][e] = al[3][e];
-                e2[1][e] = e2[2][e] * al[2][e];
-                e2[0][e] = e2[1][e] * al[1][e];
-                tot[e] = e1[3][e];
-            }
-            // across the 4 quarters of the block (a quad of lanes): exclusive prefix / suffix
-            // products of the quarter products, and exclusive prefix sums of the quarter log sums
+                // exclusive prefix of the quarter log sums across the quad, and the block total
+                float l = gl[3][e];
+                float y = __shfl_up_sync(0xffffffffu, l, 1, 4);
+                if (qq >= 1) l += y;
+                y = __shfl_up_sync(0xffffffffu, l, 2, 4);
+                if (qq >= 2) l += y;
+                y = __shfl_up_sync(0xffffffffu, l, 1, 4);
+                const float lex = qq >= 1 ? y : 0.0f;
+                Lb[e] = __shfl_sync(0xffffffffu, l, (lane & ~3) | 3);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float x = tot[e];
-                float y = __shfl_up_sync(0xffffffffu, x, 1, 4);
-                if (qq >= 1) x *= y;
-                y = __shfl_up_sync(0xffffffffu, x, 2, 4);
-                if (qq >= 2) x *= y;
-                y = __shfl_up_sync(0xffffffffu, x, 1, 4);
-                excl[e] = qq >= 1 ? y : 1.0f;
-                float z = tot[e];
-                float w = __shfl_down_sync(0xffffffffu, z, 1, 4);
-                if (qq <= 2) z *= w;
-                w = __shfl_down_sync(0xffffffffu, z, 2, 4);
-                if (qq <= 1) z *= w;
-                w = __shfl_down_sync(0xffffffffu, z, 1, 4);
-                sexc[e] = qq <= 2 ? w : 1.0f;
-                float l = Gl[3][e];
-                float m = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                if (qq >= 1) l += m;
-                m = __shfl_up_sync(0xffffffffu, l, 2, 4);
-                if (qq >= 2) l += m;
-                Lb[e] = __shfl_sync(0xffffffffu, l, (lane & ~3) | 3, 32);
-                m = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                lexc[e] = qq >= 1 ? m : 0.0f;
-            }
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    e1[s][e] *= excl[e];
-                    e2[s][e] *= sexc[e];
-                    Gl[s][e] += lexc[e];
+                for (int s = 0; s < 4; ++s) {
+                    const float G_in = gl[s][e] + lex;            // G_i - G_blockstart
+                    E1[s][e] = __expf(G_in + LN_SC);
+                    E2[s][e] = __expf(Lb[e] - G_in + LN_SC);
                 }
+            }
             if (qq == 0) {
                 const int c0 = 64 * cb + 8 * a;
 #pragma unroll
@@ -300,7 +281,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncthreads();
         {
             const int c0 = 64 * cb + 8 * a;
-            float pre[8], post[8], midF[4][8], half_lb[8];
+            // per-channel factors.  Only fM carries the 1/SC scaling (it stays a normal number);
+            // the others are <= 1 and multiply the unscaled e1 = E1/SC, e2 = E2/SC, so a
+            // product underflows only where the true value does:
+            //   fM = exp(-L_B / 2) / SC       (row exp(G_i - m_B) = E1 fM, diagonal column = E2 fM)
+            //   fG = exp(G_blockstart)        (Gamma_i = e1 fG)      fL = exp(G_C - G_blockend)
+            //   fC[I] = exp(m_I - G_blockend) for later blocks I > B (column factor = e2 fC[I])
+            float fG[8], fL[8], fM[8], fC[4][8];
             bool badB[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -317,17 +304,17 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     if (J < B) lpre += Lv[J];
                     if (J > B) lpost += Lv[J];
                 }
-                pre[e] = __expf(lpre);
-                post[e] = __expf(lpost);
+                fG[e] = __expf(lpre);
+                fL[e] = __expf(lpost);
                 badB[e] = bad[B];
-                half_lb[e] = bad[B] ? 0.0f : 0.5f * Lv[B];
+                fM[e] = __expf((bad[B] ? 0.0f : -0.5f * Lv[B]) - LN_SC);
 #pragma unroll
                 for (int I = 0; I < 4; ++I) {
                     float l = bad[I] ? 0.0f : 0.5f * Lv[I];
 #pragma unroll
                     for (int J = 0; J < 4; ++J)
                         if (J > B && J < I) l += Lv[J];
-                    midF[I][e] = I > B ? __expf(l) : 0.0f;
+                    fC[I][e] = I > B ? __expf(l) : 0.0f;
                 }
                 if (B == 0 && qq == 0) GCsm[c0 + e] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
             }
@@ -335,7 +322,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int s = 0; s < 4; ++s) {
                 const int i = 16 * B + 4 * qq + s;
                 const uint32_t off = cb * 8192 + swz(i, a);
-                float qf[8], kf[8], o[8], rf[8];
+                float qf[8], kf[8], o[8];
                 unpack8(*(const uint4 *)(stg + ST_Q + off), qf);
                 unpack8(*(const uint4 *)(stg + ST_K + off), kf);
                 // exact diagonal of P: partial q_i . k_i over this lane's 8 channels
@@ -346,42 +333,71 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 pd += __shfl_xor_sync(0xffffffffu, pd, 8);
                 pd += __shfl_xor_sync(0xffffffffu, pd, 16);
                 if (a == 0) PDsm[cb * CK + i] = pd;
-                // Q^ = Gamma q, K^ = Gamma k (in place), K~ = exp(G_C - G) k (over g)
+                float gam[8], e2s[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = qf[e] * (e1[s][e] * pre[e]);
+                for (int e = 0; e < 8; ++e) {
+                    gam[e] = (E1[s][e] * INV_SC) * fG[e];
+                    e2s[e] = E2[s][e] * INV_SC;
+                }
+                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = qf[e] * gam[e];
                 {
-                    // fp32 K-major (tf32) tile: K-block of 32 channels, two 16-byte chunks of 4
                     uint8_t *qh = sm + OFF_QH + (2 * cb + (a >> 2)) * 8192;
                     *(float4 *)(qh + swz(i, 2 * (a & 3))) = make_float4(o[0], o[1], o[2], o[3]);
                     *(float4 *)(qh + swz(i, 2 * (a & 3) + 1)) = make_float4(o[4], o[5], o[6], o[7]);
                 }
+                // K^ = Gamma k (in place), K~ = exp(G_C - G_i) k (over g)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e1[s][e] * pre[e]);
+                for (int e = 0; e < 8; ++e) o[e] = kf[e] * gam[e];
                 *(uint4 *)(stg + ST_K + off) = pack8(o);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e2[s][e] * post[e]);
+                for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e2s[e] * fL[e]);
                 *(uint4 *)(stg + ST_G + off) = pack8(o);
-                // Gram rows: [Q_B; K_B] scaled by exp(G_i - m_B) (block-start reference if bad)
+                // Gram rows [Q_B; K_B] scaled by exp(G_i - m_B) (block-start reference if bad)
+                float rf[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) rf[e] = __expf(Gl[s][e] - half_lb[e]);
+                for (int e = 0; e < 8; ++e) rf[e] = E1[s][e] * fM[e];
                 const int rq = 32 * B + 4 * qq + s;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = qf[e] * rf[e];
-                *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq, a)) = pack8(o);
+                {
+                    // hi part to the Gram rows, bf16 residual to X2 (free until the readback)
+                    const uint4 hq = pack8(o);
+                    float hf[8], lo[8];
+                    unpack8(hq, hf);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = kf[e] * rf[e];
-                *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq + 16, a)) = pack8(o);
-                // Gram columns: diagonal block exp(m_B - G_j) (0 if bad); later blocks I via e2 and
-                // the in-between block decays
+                    for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
+                    *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq, a)) = hq;
+                    *(uint4 *)(sm + OFF_X2 + cb * R_CB + swz(rq, a)) = pack8(lo);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = badB[e] ? 0.0f : kf[e] * __expf(half_lb[e] - Gl[s][e]);
-                *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(cv_start(B) + i, a)) = pack8(o);
+                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * rf[e];
+                    const uint4 hk = pack8(o);
+                    unpack8(hk, hf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
+                    *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq + 16, a)) = hk;
+                    *(uint4 *)(sm + OFF_X2 + cb * R_CB + swz(rq + 16, a)) = pack8(lo);
+                }
+                // Gram columns: diagonal block exp(m_B - G_j) (0 if bad); later blocks I
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = badB[e] ? 0.0f : kf[e] * (E2[s][e] * fM[e]);
+                {
+                    // hi part to diagonal column row i; bf16 residual over the (now dead) raw q
+                    const uint4 hc = pack8(o);
+                    float hf[8], lo[8];
+                    unpack8(hc, hf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
+                    *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(i, a)) = hc;
+                    *(uint4 *)(stg + ST_Q + off) = pack8(lo);
+                }
 #pragma unroll
                 for (int I = 1; I < 4; ++I) {
                     if (I <= B) continue;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * e2[s][e] * midF[I][e];
-                    *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(cv_start(I) + i, a)) = pack8(o);
+                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e2s[e] * fC[I][e]);
+                    *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(cv_off(I) + i, a)) = pack8(o);
                 }
             }
         }
@@ -396,6 +412,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int kk = 0; kk < 8; ++kk)
                 mma_ss(tmem + TM_G, sdesc(sR + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
                        sdesc(sCV + (kk >> 2) * CV_CB + (kk & 3) * 32, 16, 1024), id_gram, kk > 0);
+            // diagonal-block residual: R_lo x CVd (CV rows 0..63) + R x CVd_lo (over the q tile)
+            const uint32_t sRL = smem_u32(sm + OFF_X2), sCVL = smem_u32(stg + ST_Q);
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + TM_CORR, sdesc(sRL + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
+                       sdesc(sCV + (kk >> 2) * CV_CB + (kk & 3) * 32, 16, 1024), id_corr, kk > 0);
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + TM_CORR, sdesc(sR + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
+                       sdesc(sCVL + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_corr, 1);
             // O^T = S^T Q^^T at tf32: A = fp32 state in TMEM, 8 key channels per MMA
             const uint32_t sQ = smem_u32(sm + OFF_QH);
             for (int kk = 0; kk < 16; ++kk)
@@ -437,17 +461,26 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             for (int m = 0; m < I + 1; ++m) {
-                uint32_t r[8];
-                tmem_ld8(tmem + lane_q + TM_G + cv_start(I) + jbase + 8 * m, r);
-                tmem_wait_ld();
                 const int j0 = jbase + 8 * m;
+                uint32_t r[8];
+                if (j0 < 16 * I) {
+                    tmem_ld8(tmem + lane_q + TM_G + cv_off(I) + j0, r);   // earlier blocks
+                    tmem_wait_ld();
+                } else {
+                    uint32_t c8[8];                                       // own (diagonal) block
+                    tmem_ld8(tmem + lane_q + TM_G + j0, r);
+                    tmem_ld8(tmem + lane_q + TM_CORR + j0, c8);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(c8[e]));
+                }
                 float vals[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int j = j0 + e;
                     float v = __uint_as_float(r[e]);
                     const int jj = j - 16 * I;
-                    if (jj >= 0 && jj < 16) {
+                    if (nbad > 0 && jj >= 0 && jj < 16) {
 #pragma unroll
                         for (int z = 0; z < 16; ++z)
                             if (z == jj) v += corr[z];
@@ -485,6 +518,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (tid < 4) badcnt[tid] = 0;   // lists consumed
 
         // ============================================================ T = (I + A)^{-1} Diag(beta)
+        // L = I + A, blocked by 16: diagonal inverses L_II^{-1} by forward substitution
+        // (one column per thread), then A''_IK = L_II^{-1} A_IK, then block rows by distance:
+        // T_IJ = -sum_{K=J}^{I-1} A''_IK T_KJ.
         if (tid < 64) {
             const int Ib = tid >> 4, col = tid & 15;
             float x[16];
@@ -502,32 +538,42 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int r = 0; r < 16; ++r) LINV[(16 * Ib + r) * 64 + 16 * Ib + col] = x[r];
         }
         __syncthreads();
-        for (int d = 1; d < 4; ++d) {
-            float xv[3];
+        {
             const int r = tid >> 4, cc = tid & 15;
-            for (int J = 0; J + d < 4; ++J) {
-                const int I = J + d;
-                float acc = 0.0f;
-                for (int K = J; K < I; ++K)
+            float y[6];
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc += A32[(16 * I + r) * 64 + 16 * K + m] * LINV[(16 * K + m) * 64 + 16 * J + cc];
-                xv[J] = acc;
-            }
-            __syncthreads();
-            for (int J = 0; J + d < 4; ++J) LINV[(16 * (J + d) + r) * 64 + 16 * J + cc] = xv[J];
-            __syncthreads();
-            for (int J = 0; J + d < 4; ++J) {
-                const int I = J + d;
+            for (int pi = 0; pi < 6; ++pi) {
+                const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
+                const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
                 float acc = 0.0f;
 #pragma unroll
                 for (int m = 0; m < 16; ++m)
-                    if (m <= r) acc -= LINV[(16 * I + r) * 64 + 16 * I + m] * LINV[(16 * I + m) * 64 + 16 * J + cc];
-                xv[J] = acc;
+                    acc += LINV[(16 * I + r) * 64 + 16 * I + m] * A32[(16 * I + m) * 64 + 16 * K + cc];
+                y[pi] = acc;
             }
             __syncthreads();
-            for (int J = 0; J + d < 4; ++J) LINV[(16 * (J + d) + r) * 64 + 16 * J + cc] = xv[J];
+#pragma unroll
+            for (int pi = 0; pi < 6; ++pi) {
+                const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
+                const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
+                A32[(16 * I + r) * 64 + 16 * K + cc] = y[pi];
+            }
             __syncthreads();
+#pragma unroll
+            for (int d = 1; d < 4; ++d) {
+#pragma unroll
+                for (int J = 0; J + d < 4; ++J) {
+                    const int I = J + d;
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int K = J; K < I; ++K)
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            acc -= A32[(16 * I + r) * 64 + 16 * K + m] * LINV[(16 * K + m) * 64 + 16 * J + cc];
+                    LINV[(16 * I + r) * 64 + 16 * J + cc] = acc;
+                }
+                __syncthreads();
+            }
         }
         for (int idx = tid; idx < 64 * 8; idx += NT) {
             const int i = idx >> 3, jc = idx & 7;
@@ -628,20 +674,25 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mma_wait()) break;
         tc_fence_after();
         {
-            // O^T -> out (bf16), rows i < nt
+            // O^T -> bf16 tile in X2 (the load tiles' layout: 2 channel blocks of [64 rows x 128 B],
+            // 128-byte swizzle), then two TMA stores; rows past T are clipped by the tensor map
             const int v = 32 * (warp & 3) + lane;
             uint32_t r[32];
             tmem_ld32(tmem + lane_q + TM_O + 32 * half, r);
             tmem_wait_ld();
-            __nv_bfloat16 *orow = p.out + ((size_t)(b * T + t0) * p.H + h) * DD + v;
+            uint8_t *ot = sm + OFF_X2 + (v >> 6) * 8192 + ((v & 7) << 1);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * half + e;
-                if (i < nt) orow[(size_t)i * p.H * DD] = __float2bfloat16_rn(__uint_as_float(r[e]));
-            }
+            for (int e = 0; e < 32; ++e)
+                *(__nv_bfloat16 *)(ot + swz(32 * half + e, (v & 63) >> 3)) = __float2bfloat16_rn(__uint_as_float(r[e]));
         }
+        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (tid == 0) {
+            tma_store_4d(&tm_o, sm + OFF_X2, 0, h, t0, b);
+            tma_store_4d(&tm_o, sm + OFF_X2 + 8192, 64, h, t0, b);
+            bulk_commit();
+        }
     }
 
     // ---------------------------------------------------------------- final state
@@ -657,6 +708,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int e = 0; e < 32; ++e) sT[(size_t)(64 * half + cc + e) * DD + v] = __uint_as_float(r[e]);
         }
     }
+    if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -722,9 +774,10 @@ bool chunk_tc_supported(const ChunkArgs &a)
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
 {
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
-        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mg, a.g, a.B, a.T, a.H))
+        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mg, a.g, a.B, a.T, a.H) ||
+        !make_map(&mo, a.out, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -734,7 +787,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
     if (attr_err != cudaSuccess) return attr_err;
     TcParams p{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
                (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err};
-    kda_chunk_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, p);
+    kda_chunk_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();
 }
 

@@ -78,6 +78,21 @@ KDA_DEVICE void tma_load_4d(void *smem_dst, const CUtensorMap *map, int c0, int 
         : "memory");
 }
 
+// 4-D tiled store from shared memory (bulk-group completion).  Rows past the tensor's
+// extent are not written.
+KDA_DEVICE void tma_store_4d(const CUtensorMap *map, const void *smem_src, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"((uint64_t)map),
+        "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(smem_src))
+        : "memory");
+}
+KDA_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store has finished reading shared memory.
+KDA_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until every committed bulk store has completed.
+KDA_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 KDA_DEVICE void prefetch_tmap(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
