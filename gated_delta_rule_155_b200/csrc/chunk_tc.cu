@@ -74,17 +74,22 @@ constexpr int OFF_A32 = OFF_X2;                  // 16 KB fp32 [64][64]
 constexpr int OFF_LINV = OFF_X2 + 16384;         // 16 KB fp32 [64][64]
 constexpr int OFF_W = OFF_X2;                    // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
 constexpr int OFF_MISC = OFF_X2 + 32768;
-constexpr int MS_L = 0;                          // fp32 [4][128] block log-decays L_B
+constexpr int MS_BADMASK = 0;                    // uint32 [4][4]: channels with L_B < BAD_LOG, per block
 constexpr int MS_GC = 2048;                      // fp32 [128] chunk decay exp(G_C)
 constexpr int MS_BETA = 2560;                    // fp32 [64]
-constexpr int MS_BADCNT = 2816;                  // int [4]
-constexpr int MS_BADLIST = 2832;                 // uint8 [4][128]
 constexpr int MS_PD = 3344;                      // fp32 [2][64]: exact q_i . k_i halves
 constexpr int MS_BAR = 3856;                     // uint64 [3]: tma0, tma1, mma
 constexpr int MS_TSLOT = 3880;                   // uint32
 constexpr int MS_ABORT = 3884;                   // int
 constexpr int MISC_BYTES = 3904;
-constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
+// per-(block, channel) factor table, fp32 [slot][128]: fG, fL, fM, fD for blocks 0..3, then
+// fC for the six (B, I) pairs with I > B
+constexpr int FT_G = 0, FT_L = 4 * 128, FT_M = 8 * 128, FT_D = 12 * 128, FT_C = 16 * 128;
+constexpr int FT_BYTES = 22 * 128 * 4;
+constexpr int OFF_FT = OFF_MISC + MISC_BYTES;
+constexpr int SMEM_BYTES = OFF_FT + FT_BYTES + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+__host__ __device__ constexpr int fc_slot(int B, int I) { return B == 0 ? I - 1 : (B == 1 ? I + 1 : 5); }
 
 // tensor memory columns
 constexpr uint32_t TM_S = 0;     // fp32 S^T, 128 cols
@@ -128,12 +133,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *misc = sm + OFF_MISC;
-    float *Lsm = (float *)(misc + MS_L);
+    uint32_t *badmask = (uint32_t *)(misc + MS_BADMASK);
+    float *FT = (float *)(sm + OFF_FT);
     float *PDsm = (float *)(misc + MS_PD);
     float *GCsm = (float *)(misc + MS_GC);
     float *BETAsm = (float *)(misc + MS_BETA);
-    int *badcnt = (int *)(misc + MS_BADCNT);
-    uint8_t *badlist = misc + MS_BADLIST;
     uint64_t *bar_tma = (uint64_t *)(misc + MS_BAR);
     uint64_t *bar_mma = bar_tma + 2;
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
@@ -153,7 +157,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&bar_tma[1], 1);
         mbar_init(bar_mma, 1);
         *abort_flag = 0;
-        for (int i = 0; i < 4; ++i) badcnt[i] = 0;
+        for (int i = 0; i < 16; ++i) badmask[i] = 0u;
         fence_mbar_init();
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_g);
         prefetch_tmap(&tm_o);
@@ -211,6 +215,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t id_op = idesc_bf16(128, 64, false, false);
     const uint32_t id_s = idesc_bf16(128, 128, false, true);
 
+    // beta of the next chunk is loaded one chunk ahead, so its global-memory latency never
+    // sits on the path into prep
+    auto load_beta = [&](int n) -> float {
+        const int t = n * CK + tid;
+        return (tid < CK && t < T) ? __bfloat162float(p.beta[(size_t)(b * T + t) * p.H + h]) : 0.0f;
+    };
+    float beta_next = nchunks > 0 ? load_beta(0) : 0.0f;
+
     for (int n = 0; n < nchunks; ++n) {
         const int X = n & 1;
         uint8_t *stg = sm + (X ? OFF_REG1 : OFF_REG0);
@@ -224,105 +236,108 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err)) break;
 
         // ============================================================ prep
-        if (tid < CK) BETAsm[tid] = tid < nt ? __bfloat162float(p.beta[(size_t)(b * T + t0 + tid) * p.H + h]) : 0.0f;
-        const int B = warp & 3;           // token block of this warp
-        const int cb = warp >> 2;         // channel block (64 channels)
-        const int qq = lane & 3;          // token quarter inside the block
-        const int a = lane >> 2;          // 16-byte chunk (8 channels) inside the channel block
-        // per (token s of this lane's quarter, channel e of its 8), with SC = 2^120:
-        //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
-        //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
-        // formed from log-domain prefix sums (no partial product can underflow); both are
-        // normal numbers for block log-decays down to -168 (SC e^-168 ~ e^-84.8), so the
-        // midpoint factors below are per-channel constants times E1 or E2.
-        constexpr float INV_SC = 7.523164e-37f;    // 2^-120
+        if (tid < CK) BETAsm[tid] = beta_next;
+        beta_next = n + 1 < nchunks ? load_beta(n + 1) : 0.0f;
+        constexpr float INV_SC = 7.523164e-37f;    // SC = 2^120, INV_SC = 2^-120
         constexpr float LN_SC = 83.17766f;         // 120 ln 2
-        float E1[4][8], E2[4][8], Lb[8];
+        // pass 1: block log-decays L_B (sum of g over a 16-token block) per channel, and from
+        // them the per-(block, channel) factor table, computed once per chunk:
+        //   fG = exp(G_blockstart)      fL = exp(G_C - G_blockend)
+        //   fM = exp(-L_B / 2) / SC     (block-start reference, 1 / SC, where L_B < BAD_LOG)
+        //   fD = fM, or 0 where L_B < BAD_LOG (those diagonal terms are added exactly later)
+        //   fC(B, I) = exp(m_I - G_blockend of B) for later blocks I > B, m_I the reference of I
+        // All exponents are sums of non-positive log-decays (plus L_B / 2 >= -84 for fM), so a
+        // factor underflows only where the exact value does.
         {
-            float gl[4][8];
+            const int c = tid >> 1, par = tid & 1;     // channel; blocks 2 par and 2 par + 1
+            const uint8_t *gcol = stg + ST_G + (c >> 6) * 8192 + ((c & 7) << 1);
+            const int chk = (c & 63) >> 3;
+            float Ls[2];
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int i = 16 * B + 4 * qq + s;
-                float gf[8];
-                unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), gf);
+            for (int u = 0; u < 2; ++u) {
+                float acc = 0.0f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) gl[s][e] = (s == 0 ? 0.0f : gl[s - 1][e]) + gf[e];
+                for (int t = 0; t < 16; ++t)
+                    acc += __bfloat162float(*(const __nv_bfloat16 *)(gcol + swz(16 * (2 * par + u) + t, chk)));
+                Ls[u] = acc;
             }
+            const float x0 = __shfl_xor_sync(0xffffffffu, Ls[0], 1), x1 = __shfl_xor_sync(0xffffffffu, Ls[1], 1);
+            const float Lv[4] = {par ? x0 : Ls[0], par ? x1 : Ls[1], par ? Ls[0] : x0, par ? Ls[1] : x1};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                // exclusive prefix of the quarter log sums across the quad, and the block total
-                float l = gl[3][e];
-                float y = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                if (qq >= 1) l += y;
-                y = __shfl_up_sync(0xffffffffu, l, 2, 4);
-                if (qq >= 2) l += y;
-                y = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                const float lex = qq >= 1 ? y : 0.0f;
-                Lb[e] = __shfl_sync(0xffffffffu, l, (lane & ~3) | 3);
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const float G_in = gl[s][e] + lex;            // G_i - G_blockstart
-                    E1[s][e] = __expf(G_in + LN_SC);
-                    E2[s][e] = __expf(Lb[e] - G_in + LN_SC);
-                }
-            }
-            if (qq == 0) {
-                const int c0 = 64 * cb + 8 * a;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    Lsm[B * DD + c0 + e] = Lb[e];
-                    if (!(Lb[e] >= BAD_LOG)) {
-                        const int slot = atomicAdd(&badcnt[B], 1);
-                        badlist[B * DD + slot] = (uint8_t)(c0 + e);
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        {
-            const int c0 = 64 * cb + 8 * a;
-            // per-channel factors.  Only fM carries the 1/SC scaling (it stays a normal number);
-            // the others are <= 1 and multiply the unscaled e1 = E1/SC, e2 = E2/SC, so a
-            // product underflows only where the true value does:
-            //   fM = exp(-L_B / 2) / SC       (row exp(G_i - m_B) = E1 fM, diagonal column = E2 fM)
-            //   fG = exp(G_blockstart)        (Gamma_i = e1 fG)      fL = exp(G_C - G_blockend)
-            //   fC[I] = exp(m_I - G_blockend) for later blocks I > B (column factor = e2 fC[I])
-            float fG[8], fL[8], fM[8], fC[4][8];
-            bool badB[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                float Lv[4];
-                bool bad[4];
-#pragma unroll
-                for (int J = 0; J < 4; ++J) {
-                    Lv[J] = Lsm[J * DD + c0 + e];
-                    bad[J] = !(Lv[J] >= BAD_LOG);
-                }
+            for (int u = 0; u < 2; ++u) {
+                const int Bq = 2 * par + u;
                 float lpre = 0.0f, lpost = 0.0f;
 #pragma unroll
                 for (int J = 0; J < 4; ++J) {
-                    if (J < B) lpre += Lv[J];
-                    if (J > B) lpost += Lv[J];
+                    if (J < Bq) lpre += Lv[J];
+                    if (J > Bq) lpost += Lv[J];
                 }
-                fG[e] = __expf(lpre);
-                fL[e] = __expf(lpost);
-                badB[e] = bad[B];
-                fM[e] = __expf((bad[B] ? 0.0f : -0.5f * Lv[B]) - LN_SC);
+                const bool badB = !(Ls[u] >= BAD_LOG);
+                const float fM = __expf((badB ? 0.0f : -0.5f * Ls[u]) - LN_SC);
+                FT[FT_G + Bq * DD + c] = __expf(lpre);
+                FT[FT_L + Bq * DD + c] = __expf(lpost);
+                FT[FT_M + Bq * DD + c] = fM;
+                FT[FT_D + Bq * DD + c] = badB ? 0.0f : fM;
+                if (badB) atomicOr(&badmask[Bq * 4 + (c >> 5)], 1u << (c & 31));
 #pragma unroll
-                for (int I = 0; I < 4; ++I) {
-                    float l = bad[I] ? 0.0f : 0.5f * Lv[I];
+                for (int I = 1; I < 4; ++I) {
+                    if (I <= Bq) continue;
+                    float l = Lv[I] >= BAD_LOG ? 0.5f * Lv[I] : 0.0f;
 #pragma unroll
-                    for (int J = 0; J < 4; ++J)
-                        if (J > B && J < I) l += Lv[J];
-                    fC[I][e] = I > B ? __expf(l) : 0.0f;
+                    for (int J = 1; J < 3; ++J)
+                        if (J > Bq && J < I) l += Lv[J];
+                    FT[FT_C + fc_slot(Bq, I) * DD + c] = __expf(l);
                 }
-                if (B == 0 && qq == 0) GCsm[c0 + e] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
             }
+            if (par == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
+        }
+        __syncthreads();
+        // pass 2: per token.  Lane (qq, a) of warp (B, cb) takes tokens 16 B + 4 qq + s, s < 4,
+        // and channels c0 .. c0 + 7.  With SC = 2^120:
+        //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
+        //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
+        // from log-domain prefix sums, so no partial product can underflow; both are normal
+        // numbers for block log-decays down to BAD_LOG (SC e^-168 ~ e^-84.8).
+        {
+            const int B = warp & 3;           // token block of this warp
+            const int cb = warp >> 2;         // channel block (64 channels)
+            const int qq = lane & 3;          // token quarter inside the block
+            const int a = lane >> 2;          // 16-byte chunk (8 channels) inside the channel block
+            const int c0 = 64 * cb + 8 * a;
+            float Gin[4][8], Lb[8];
+            {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const int i = 16 * B + 4 * qq + s;
+                    float gf[8];
+                    unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), gf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) Gin[s][e] = (s == 0 ? 0.0f : Gin[s - 1][e]) + gf[e];
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    // exclusive prefix of the quarter log sums across the quad, and the block total
+                    float l = Gin[3][e];
+                    float y = __shfl_up_sync(0xffffffffu, l, 1, 4);
+                    if (qq >= 1) l += y;
+                    y = __shfl_up_sync(0xffffffffu, l, 2, 4);
+                    if (qq >= 2) l += y;
+                    y = __shfl_up_sync(0xffffffffu, l, 1, 4);
+                    const float lex = qq >= 1 ? y : 0.0f;
+                    Lb[e] = __shfl_sync(0xffffffffu, l, (lane & ~3) | 3);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) Gin[s][e] += lex;   // G_i - G_blockstart
+                }
+            }
+            auto ftab = [&](int off, float (&f)[8]) {
+                const float4 u0 = *(const float4 *)(FT + off + c0), u1 = *(const float4 *)(FT + off + c0 + 4);
+                f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+            };
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const int i = 16 * B + 4 * qq + s;
                 const uint32_t off = cb * 8192 + swz(i, a);
-                float qf[8], kf[8], o[8];
+                float qf[8], kf[8], o[8], E1[8], E2[8], f[8];
                 unpack8(*(const uint4 *)(stg + ST_Q + off), qf);
                 unpack8(*(const uint4 *)(stg + ST_K + off), kf);
                 // exact diagonal of P: partial q_i . k_i over this lane's 8 channels
@@ -333,38 +348,49 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 pd += __shfl_xor_sync(0xffffffffu, pd, 8);
                 pd += __shfl_xor_sync(0xffffffffu, pd, 16);
                 if (a == 0) PDsm[cb * CK + i] = pd;
-                float gam[8], e2s[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    gam[e] = (E1[s][e] * INV_SC) * fG[e];
-                    e2s[e] = E2[s][e] * INV_SC;
+                    E1[e] = __expf(Gin[s][e] + LN_SC);
+                    E2[e] = __expf(Lb[e] - Gin[s][e] + LN_SC);
                 }
-                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA)
+                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA), Gamma_i = (E1 / SC) fG;
+                // odd quarters write their two 16-byte halves in the other order, which spreads
+                // each store over all 32 banks
+                ftab(FT_G + B * DD, f);
+                float gam[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = qf[e] * gam[e];
+                for (int e = 0; e < 8; ++e) {
+                    gam[e] = (E1[e] * INV_SC) * f[e];
+                    o[e] = qf[e] * gam[e];
+                }
                 {
                     uint8_t *qh = sm + OFF_QH + (2 * cb + (a >> 2)) * 8192;
-                    *(float4 *)(qh + swz(i, 2 * (a & 3))) = make_float4(o[0], o[1], o[2], o[3]);
-                    *(float4 *)(qh + swz(i, 2 * (a & 3) + 1)) = make_float4(o[4], o[5], o[6], o[7]);
+                    const bool sw = qq & 1;
+                    const float4 lo4 = make_float4(o[0], o[1], o[2], o[3]), hi4 = make_float4(o[4], o[5], o[6], o[7]);
+                    *(float4 *)(qh + swz(i, 2 * (a & 3) + (sw ? 1 : 0))) = sw ? hi4 : lo4;
+                    *(float4 *)(qh + swz(i, 2 * (a & 3) + (sw ? 0 : 1))) = sw ? lo4 : hi4;
                 }
-                // K^ = Gamma k (in place), K~ = exp(G_C - G_i) k (over g)
+                // K^ = Gamma k (in place)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * gam[e];
                 *(uint4 *)(stg + ST_K + off) = pack8(o);
+                // K~ = exp(G_C - G_i) k (over g) = k (E2 / SC) fL
+                ftab(FT_L + B * DD, f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e2s[e] * fL[e]);
+                for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
                 *(uint4 *)(stg + ST_G + off) = pack8(o);
-                // Gram rows [Q_B; K_B] scaled by exp(G_i - m_B) (block-start reference if bad)
-                float rf[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) rf[e] = E1[s][e] * fM[e];
+                // Gram rows [Q_B; K_B] scaled by E1 fM = exp(G_i - m_B): hi part to the Gram
+                // rows, bf16 residual to X2 (free until the readback)
+                ftab(FT_M + B * DD, f);
                 const int rq = 32 * B + 4 * qq + s;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = qf[e] * rf[e];
                 {
-                    // hi part to the Gram rows, bf16 residual to X2 (free until the readback)
+                    float rf[8], hf[8], lo[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        rf[e] = E1[e] * f[e];
+                        o[e] = qf[e] * rf[e];
+                    }
                     const uint4 hq = pack8(o);
-                    float hf[8], lo[8];
                     unpack8(hq, hf);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
@@ -379,24 +405,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq + 16, a)) = hk;
                     *(uint4 *)(sm + OFF_X2 + cb * R_CB + swz(rq + 16, a)) = pack8(lo);
                 }
-                // Gram columns: diagonal block exp(m_B - G_j) (0 if bad); later blocks I
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = badB[e] ? 0.0f : kf[e] * (E2[s][e] * fM[e]);
+                // Gram columns, diagonal block: k E2 fD = k exp(m_B - G_j) (0 where L_B < BAD_LOG);
+                // hi part to diagonal column row i, bf16 residual over the (now dead) raw q
+                ftab(FT_D + B * DD, f);
                 {
-                    // hi part to diagonal column row i; bf16 residual over the (now dead) raw q
-                    const uint4 hc = pack8(o);
                     float hf[8], lo[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * (E2[e] * f[e]);
+                    const uint4 hc = pack8(o);
                     unpack8(hc, hf);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
                     *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(i, a)) = hc;
                     *(uint4 *)(stg + ST_Q + off) = pack8(lo);
                 }
+                // Gram columns for later blocks I > B: k (E2 / SC) fC(B, I)
 #pragma unroll
                 for (int I = 1; I < 4; ++I) {
                     if (I <= B) continue;
+                    ftab(FT_C + fc_slot(B, I) * DD, f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * (e2s[e] * fC[I][e]);
+                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
                     *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(cv_off(I) + i, a)) = pack8(o);
                 }
             }
@@ -440,51 +469,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int jbase = half * ncol;
             const float bi = BETAsm[i];
             const float pdiag = PDsm[i] + PDsm[CK + i];   // exact q_i . k_i
-            // exact diagonal-block contributions of channels whose block decay underflows
-            float corr[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) corr[e] = 0.0f;
-            const int nbad = badcnt[I];
-            for (int u = 0; u < nbad; ++u) {
-                const int c = badlist[I * DD + u];
-                const size_t rowi = ((size_t)(b * T + t0 + i) * p.H + h) * DD + c;
-                const float xi = (t0 + i < T) ? __bfloat162float((is_q ? p.q : p.k)[rowi]) : 0.0f;
-                float w = 1.0f;
-                for (int jj = i - 16 * I; jj >= 0; --jj) {
-                    const int j = 16 * I + jj;
-                    const bool valid = t0 + j < T;
-                    const size_t rowj = ((size_t)(b * T + t0 + j) * p.H + h) * DD + c;
-                    const float kj = valid ? __bfloat162float(p.k[rowj]) : 0.0f;
-                    corr[jj] += xi * kj * w;
-                    const float gj = valid ? __bfloat162float(p.g[rowj]) : 0.0f;
-                    w *= __expf(gj);
-                }
-            }
-            for (int m = 0; m < I + 1; ++m) {
-                const int j0 = jbase + 8 * m;
-                uint32_t r[8];
-                if (j0 < 16 * I) {
-                    tmem_ld8(tmem + lane_q + TM_G + cv_off(I) + j0, r);   // earlier blocks
-                    tmem_wait_ld();
-                } else {
-                    uint32_t c8[8];                                       // own (diagonal) block
-                    tmem_ld8(tmem + lane_q + TM_G + j0, r);
-                    tmem_ld8(tmem + lane_q + TM_CORR + j0, c8);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) + __uint_as_float(c8[e]));
-                }
+            const uint32_t *bmask = badmask + 4 * I;
+            // the warp's TMEM loads go out in two batches (earlier-block columns, then the
+            // diagonal block with its residual), one wait each; chunks are counted from the
+            // warp's last 8 columns, so only mm = 0, 1 can be diagonal
+            auto emit = [&](int j0, const uint32_t (&r)[8]) {
                 float vals[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int j = j0 + e;
-                    float v = __uint_as_float(r[e]);
-                    const int jj = j - 16 * I;
-                    if (nbad > 0 && jj >= 0 && jj < 16) {
-#pragma unroll
-                        for (int z = 0; z < 16; ++z)
-                            if (z == jj) v += corr[z];
-                    }
+                    const float v = __uint_as_float(r[e]);
                     if (is_q) vals[e] = j < i ? v : (j == i ? pdiag : 0.0f);
                     else vals[e] = j < i ? bi * v : 0.0f;
                 }
@@ -501,6 +495,70 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     *(float4 *)(A32 + i * 64 + j0) = make_float4(vals[0], vals[1], vals[2], vals[3]);
                     *(float4 *)(A32 + i * 64 + j0 + 4) = make_float4(vals[4], vals[5], vals[6], vals[7]);
                 }
+            };
+            {
+                uint32_t r[4][8];
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const int j0 = jbase + 8 * (I - mm);
+                    if (mm <= I && j0 < 16 * I) tmem_ld8(tmem + lane_q + TM_G + cv_off(I) + j0, r[mm]);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const int j0 = jbase + 8 * (I - mm);
+                    if (mm <= I && j0 < 16 * I) emit(j0, r[mm]);
+                }
+            }
+            {
+                uint32_t r[2][8], c8[2][8];
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    const int j0 = jbase + 8 * (I - mm);
+                    if (mm <= I && j0 >= 16 * I) {
+                        tmem_ld8(tmem + lane_q + TM_G + j0, r[mm]);
+                        tmem_ld8(tmem + lane_q + TM_CORR + j0, c8[mm]);
+                    }
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int mm = 0; mm < 2; ++mm) {
+                    const int j0 = jbase + 8 * (I - mm);
+                    if (mm <= I && j0 >= 16 * I) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            r[mm][e] = __float_as_uint(__uint_as_float(r[mm][e]) + __uint_as_float(c8[mm][e]));
+                        emit(j0, r[mm]);
+                    }
+                }
+            }
+            // exact diagonal-block terms of channels whose block decay underflows the Gram
+            // factorisation, added in place to this thread's own entries (rare path)
+            for (int wd = 0; wd < 4; ++wd) {
+                for (uint32_t m = bmask[wd]; m != 0u; m &= m - 1u) {
+                    const int c = 32 * wd + __ffs((int)m) - 1;
+                    const size_t rowi = ((size_t)(b * T + t0 + i) * p.H + h) * DD + c;
+                    const float xi = (t0 + i < T) ? __bfloat162float((is_q ? p.q : p.k)[rowi]) : 0.0f;
+                    float w = 1.0f;   // exp(G_i - G_j), built backwards from j = i
+                    for (int j = i; j >= 16 * I; --j) {
+                        const bool valid = t0 + j < T;
+                        const size_t rowj = ((size_t)(b * T + t0 + j) * p.H + h) * DD + c;
+                        if (j < i && j >= jbase && j < jbase + ncol) {
+                            const float d = xi * (valid ? __bfloat162float(p.k[rowj]) : 0.0f) * w;
+                            if (is_q) {
+                                __nv_bfloat16 *ph = (__nv_bfloat16 *)(sm + OFF_P + swz(i, j >> 3)) + (j & 7);
+                                __nv_bfloat16 *pl = (__nv_bfloat16 *)(sm + OFF_PL + swz(i, j >> 3)) + (j & 7);
+                                const float v = __bfloat162float(*ph) + __bfloat162float(*pl) + d;
+                                const __nv_bfloat16 vh = __float2bfloat16_rn(v);
+                                *ph = vh;
+                                *pl = __float2bfloat16_rn(v - __bfloat162float(vh));
+                            } else {
+                                A32[i * 64 + j] += bi * d;
+                            }
+                        }
+                        w *= __expf(valid ? __bfloat162float(p.g[rowj]) : 0.0f);
+                    }
+                }
             }
             if (half == 1) {
                 for (int jc = 2 * (I + 1); jc < 8; ++jc) {
@@ -515,62 +573,80 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncthreads();
-        if (tid < 4) badcnt[tid] = 0;   // lists consumed
+        if (tid < 16) badmask[tid] = 0u;   // masks consumed
 
         // ============================================================ T = (I + A)^{-1} Diag(beta)
-        // L = I + A, blocked by 16: diagonal inverses L_II^{-1} by forward substitution
-        // (one column per thread), then A''_IK = L_II^{-1} A_IK, then block rows by distance:
-        // T_IJ = -sum_{K=J}^{I-1} A''_IK T_KJ.
+        // L = I + A, blocked by 16: diagonal inverses L_II^{-1} (right-looking forward
+        // substitution, one column per thread), then A''_IK = L_II^{-1} A_IK, then block rows
+        // by distance: T_IJ = -sum_{K=J}^{I-1} A''_IK T_KJ.  The block products run on
+        // strips of 4 rows x 1 column per thread (row segments read as float4).
         if (tid < 64) {
             const int Ib = tid >> 4, col = tid & 15;
+            const float *Ab = A32 + (16 * Ib) * 64 + 16 * Ib;
             float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = (r == col) ? 1.0f : 0.0f;
-                if (r > col) {
+            for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.0f : 0.0f;
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        if (m >= col && m < r) acc -= A32[(16 * Ib + r) * 64 + 16 * Ib + m] * x[m];
-                }
-                x[r] = r >= col ? acc : 0.0f;
-            }
+            for (int m = 0; m < 15; ++m)
+#pragma unroll
+                for (int r = m + 1; r < 16; ++r) x[r] -= Ab[r * 64 + m] * x[m];
 #pragma unroll
             for (int r = 0; r < 16; ++r) LINV[(16 * Ib + r) * 64 + 16 * Ib + col] = x[r];
         }
         __syncthreads();
         {
-            const int r = tid >> 4, cc = tid & 15;
-            float y[6];
+            const int set = tid >> 6;               // which block product this thread serves
+            const int r0 = ((tid >> 4) & 3) * 4;    // rows r0..r0+3 of the 16x16 block
+            const int cc = tid & 15;                // column
+            // acc[q] += sum_m X[rowbase + r0 + q][colX + m] * Y[rowY + m][colY + cc]
+            auto strip = [&](const float *X, int xrow, int xcol, const float *Y, int yrow, int ycol,
+                             float (&acc)[4]) {
 #pragma unroll
-            for (int pi = 0; pi < 6; ++pi) {
-                const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
-                const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
-                float acc = 0.0f;
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float y0 = Y[(yrow + m4 + 0) * 64 + ycol + cc], y1 = Y[(yrow + m4 + 1) * 64 + ycol + cc];
+                    const float y2 = Y[(yrow + m4 + 2) * 64 + ycol + cc], y3 = Y[(yrow + m4 + 3) * 64 + ycol + cc];
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc += LINV[(16 * I + r) * 64 + 16 * I + m] * A32[(16 * I + m) * 64 + 16 * K + cc];
-                y[pi] = acc;
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 xv = *(const float4 *)(X + (xrow + r0 + q) * 64 + xcol + m4);
+                        acc[q] += xv.x * y0 + xv.y * y1 + xv.z * y2 + xv.w * y3;
+                    }
+                }
+            };
+            // A''_IK for the 6 pairs (I, K), K < I: sets 0..3 take pairs {set, set + 4}
+            float y[2][4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int pi = set + 4 * u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) y[u][q] = 0.0f;
+                if (pi < 6) {
+                    const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
+                    const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
+                    strip(LINV, 16 * I, 16 * I, A32, 16 * I, 16 * K, y[u]);
+                }
             }
             __syncthreads();
 #pragma unroll
-            for (int pi = 0; pi < 6; ++pi) {
-                const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
-                const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
-                A32[(16 * I + r) * 64 + 16 * K + cc] = y[pi];
+            for (int u = 0; u < 2; ++u) {
+                const int pi = set + 4 * u;
+                if (pi < 6) {
+                    const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
+                    const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) A32[(16 * I + r0 + q) * 64 + 16 * K + cc] = y[u][q];
+                }
             }
             __syncthreads();
 #pragma unroll
             for (int d = 1; d < 4; ++d) {
+                const int J = set, I = set + d;
+                if (I < 4) {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int J = 0; J + d < 4; ++J) {
-                    const int I = J + d;
-                    float acc = 0.0f;
+                    for (int K = 0; K < 3; ++K)
+                        if (K >= J && K < I) strip(A32, 16 * I, 16 * K, LINV, 16 * K, 16 * J, acc);
 #pragma unroll
-                    for (int K = J; K < I; ++K)
-#pragma unroll
-                        for (int m = 0; m < 16; ++m)
-                            acc -= A32[(16 * I + r) * 64 + 16 * K + m] * LINV[(16 * K + m) * 64 + 16 * J + cc];
-                    LINV[(16 * I + r) * 64 + 16 * J + cc] = acc;
+                    for (int q = 0; q < 4; ++q) LINV[(16 * I + r0 + q) * 64 + 16 * J + cc] = -acc[q];
                 }
                 __syncthreads();
             }
