@@ -49,7 +49,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int NT = 256;       // threads
+constexpr int NT = 512;       // threads: 16 warps = 4 TMEM lane quarters x 4 column groups
 constexpr int CK = 64;        // chunk
 constexpr int DD = 128;       // dk = dv
 constexpr float BAD_LOG = -168.0f;  // block log-decays below this take the exact fallback
@@ -62,34 +62,48 @@ constexpr int ST_Q = 0, ST_K = 16384, ST_V = 32768, ST_G = 49152;     // inside 
 constexpr int GR_R = 0, GR_CV = 32768;                                // inside a Gram region
 constexpr int R_CB = 16384;                      // R: 128 rows x 128 B per channel block
 constexpr int CV_ROWS = 160, CV_CB = CV_ROWS * 128;
-// X1 (32 KB): Q^ in fp32 (tf32 K-major [i][c], prep -> O init); then P, P_lo, T (bf16)
-// X2 (32 KB): A and L^{-1} in fp32 (inverse); then W in fp32 (tf32 K-major [i][c])
+// X1 (32 KB): Q^ in fp32 (tf32 K-major [i][c]), from prep until the O-init MMA (issued
+// after the Gram readback) has run
+// X2 (32 KB): R_lo (prep -> Gram); A and L^{-1} in fp32 (inverse); W in fp32 (tf32 K-major
+// [i][c]); the O tile
+// P and P_lo (bf16 K-major [i][j], 8 KB each) take the stage's q tile once the Gram MMAs have
+// read the residual columns kept there; T (bf16 K-major [i][j], 8 KB) sits in the factor table
 constexpr int OFF_X1 = 2 * REG_BYTES;
 constexpr int OFF_QH = OFF_X1;                   // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
-constexpr int OFF_P = OFF_X1;                    // 8 KB bf16 K-major [i][j]: P (hi part)
-constexpr int OFF_PL = OFF_P + 8192;             // 8 KB bf16: P - P_hi (lo part)
-constexpr int OFF_T = OFF_PL + 8192;             // 8 KB bf16 K-major [i][j]
+constexpr int ST_P = ST_Q, ST_PL = ST_Q + 8192;  // inside the stage region
 constexpr int OFF_X2 = OFF_X1 + 32768;
-constexpr int OFF_A32 = OFF_X2;                  // 16 KB fp32 [64][64]
-constexpr int OFF_LINV = OFF_X2 + 16384;         // 16 KB fp32 [64][64]
+// A and L^{-1}: fp32 [64][AST]; the row stride of 68 floats shifts consecutive rows by four
+// banks, so column reads and row-segment writes spread over all banks.  L^{-1} runs 2 KB past
+// X2 into the factor table, which is dead between prep and the next chunk.
+constexpr int AST = 68;
+constexpr int OFF_A32 = OFF_X2;
+constexpr int OFF_LINV = OFF_X2 + 64 * AST * 4;
 constexpr int OFF_W = OFF_X2;                    // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
-constexpr int OFF_MISC = OFF_X2 + 32768;
+// per-(block, channel) table, fp32 rows of FSTRIDE (128 channels + padding that puts the
+// four blocks of one channel in different banks): fG, fL, fM, block log-decay L_B and
+// first-half log-decay H_B (tokens 0..7 of the block) for blocks 0..3, then fC for the six
+// (B, I) pairs with I > B
+constexpr int FSTRIDE = 136;
+constexpr int FT_G = 0, FT_L = 4, FT_M = 8, FT_LB = 12, FT_H8 = 16, FT_C = 20;   // row numbers
+constexpr int FT_BYTES = 26 * FSTRIDE * 4;
+constexpr int OFF_FT = OFF_X2 + 32768;
+constexpr int OFF_T = OFF_FT + 2048;             // past L^{-1}'s overhang, 1024-aligned
+constexpr int OFF_MISC = OFF_FT + FT_BYTES;
 constexpr int MS_BADMASK = 0;                    // uint32 [4][4]: channels with L_B < BAD_LOG, per block
-constexpr int MS_GC = 2048;                      // fp32 [128] chunk decay exp(G_C)
-constexpr int MS_BETA = 2560;                    // fp32 [64]
-constexpr int MS_PD = 3344;                      // fp32 [2][64]: exact q_i . k_i halves
-constexpr int MS_BAR = 3856;                     // uint64 [3]: tma0, tma1, mma
-constexpr int MS_TSLOT = 3880;                   // uint32
-constexpr int MS_ABORT = 3884;                   // int
-constexpr int MISC_BYTES = 3904;
-// per-(block, channel) factor table, fp32 [slot][128]: fG, fL, fM, fD for blocks 0..3, then
-// fC for the six (B, I) pairs with I > B
-constexpr int FT_G = 0, FT_L = 4 * 128, FT_M = 8 * 128, FT_D = 12 * 128, FT_C = 16 * 128;
-constexpr int FT_BYTES = 22 * 128 * 4;
-constexpr int OFF_FT = OFF_MISC + MISC_BYTES;
-constexpr int SMEM_BYTES = OFF_FT + FT_BYTES + 1024;  // + alignment slack
+constexpr int MS_GC = 64;                        // fp32 [128] chunk decay exp(G_C)
+constexpr int MS_BETA = 576;                     // fp32 [64]
+constexpr int MS_PD = 832;                       // fp32 [4][64]: exact q_i . k_i, per channel quarter
+constexpr int MS_BAR = 1856;                     // uint64 [4]: tma0, tma1, mma, O init
+constexpr int MS_TSLOT = 1888;                   // uint32
+constexpr int MS_ABORT = 1892;                   // int
+constexpr int MS_BRAW = 1920;                    // uint32 [2][64]: beta words in flight (cp.async)
+constexpr int MISC_BYTES = 2432;
+constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+static_assert(OFF_LINV + 64 * AST * 4 <= OFF_MISC, "L^{-1} stays clear of the barriers");
+static_assert(OFF_MISC % 16 == 0 && OFF_FT % 16 == 0 && OFF_T % 1024 == 0 && OFF_T + 8192 <= OFF_MISC, "alignment");
 __host__ __device__ constexpr int fc_slot(int B, int I) { return B == 0 ? I - 1 : (B == 1 ? I + 1 : 5); }
+KDA_DEVICE int aidx(int i, int j) { return i * AST + j; }
 
 // tensor memory columns
 constexpr uint32_t TM_S = 0;     // fp32 S^T, 128 cols
@@ -138,8 +152,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float *PDsm = (float *)(misc + MS_PD);
     float *GCsm = (float *)(misc + MS_GC);
     float *BETAsm = (float *)(misc + MS_BETA);
+    uint32_t *BRAW = (uint32_t *)(misc + MS_BRAW);
     uint64_t *bar_tma = (uint64_t *)(misc + MS_BAR);
     uint64_t *bar_mma = bar_tma + 2;
+    uint64_t *bar_o = bar_tma + 3;
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
     float *A32 = (float *)(sm + OFF_A32);
@@ -149,13 +165,16 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
     const int T = p.T;
     const int nchunks = (T + CK - 1) / CK;
-    const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lane quarter
-    const int half = warp >> 2;
+    // a warp reaches TMEM lanes 32 (warp & 3) .. + 31; the four warps of a lane quarter split
+    // the columns of every TMEM tile they read or write into column groups cg = warp >> 2
+    const int lq = warp & 3, cg = warp >> 2;
+    const uint32_t lane_q = (uint32_t)(32 * lq) << 16;
 
     if (tid == 0) {
         mbar_init(&bar_tma[0], 1);
         mbar_init(&bar_tma[1], 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_o, 1);
         *abort_flag = 0;
         for (int i = 0; i < 16; ++i) badmask[i] = 0u;
         fence_mbar_init();
@@ -187,16 +206,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     // ---------------------------------------------------------------- initial state
     {
-        const int v = 32 * (warp & 3) + lane;
+        // S^T: lane v = value column, TMEM column c = key channel
+        const int v = 32 * lq + lane;
         const float *s0 = p.s0 ? p.s0 + (size_t)bh * DD * DD : nullptr;
-        for (int cc = 0; cc < 64; cc += 32) {
-            uint32_t r[32];
-            for (int e = 0; e < 32; ++e) {
-                const int c = 64 * half + cc + e;
-                r[e] = __float_as_uint(s0 ? s0[(size_t)c * DD + v] : 0.0f);
-            }
-            tmem_st32(tmem + lane_q + TM_S + 64 * half + cc, r);
-        }
+        uint32_t r[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(s0 ? s0[(size_t)(32 * cg + e) * DD + v] : 0.0f);
+        tmem_st32(tmem + lane_q + TM_S + 32 * cg, r);
         tmem_wait_st();
     }
 
@@ -207,156 +223,166 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return ok;
     };
 
-    const uint32_t id_gram = idesc_bf16(128, CV_ROWS, false, false);
-    const uint32_t id_corr = idesc_bf16(128, 64, false, false);
-    const uint32_t id_o0 = idesc_tf32(128, 64, false, false);
-    const uint32_t id_wt = idesc_bf16(128, 64, true, false);
-    const uint32_t id_u = idesc_tf32(128, 64, false, false, true);
-    const uint32_t id_op = idesc_bf16(128, 64, false, false);
-    const uint32_t id_s = idesc_bf16(128, 128, false, true);
+    constexpr uint32_t id_gram = idesc_bf16(128, CV_ROWS, false, false);
+    constexpr uint32_t id_corr = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id_o0 = idesc_tf32(128, 64, false, false);
+    constexpr uint32_t id_wt = idesc_bf16(128, 64, true, false);
+    constexpr uint32_t id_u = idesc_tf32(128, 64, false, false, true);
+    constexpr uint32_t id_op = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
 
-    // beta of the next chunk is loaded one chunk ahead, so its global-memory latency never
-    // sits on the path into prep
-    auto load_beta = [&](int n) -> float {
-        const int t = n * CK + tid;
-        return (tid < CK && t < T) ? __bfloat162float(p.beta[(size_t)(b * T + t) * p.H + h]) : 0.0f;
+    // beta of the next chunk is copied one chunk ahead, global -> shared by cp.async, so no
+    // thread ever waits on its memory latency: the aligned 32-bit word that holds beta_t
+    // (2 bytes of it when beta_t is the word's low half, which may be the last element)
+    auto beta_async = [&](int nn) {   // tid < CK
+        const int t = nn * CK + tid;
+        const void *src = p.beta;
+        uint32_t bytes = 0;
+        if (t < T) {
+            const uintptr_t ea = (uintptr_t)(p.beta + (size_t)(b * T + t) * p.H + h);
+            bytes = (ea & 2) ? 4u : 2u;
+            src = (const void *)(ea & ~(uintptr_t)3);
+        }
+        cp_async4(smem_u32(BRAW + (nn & 1) * CK + tid), src, bytes);
+        cp_async_commit();
     };
-    float beta_next = nchunks > 0 ? load_beta(0) : 0.0f;
+    if (tid < CK && nchunks > 0) beta_async(0);
 
     for (int n = 0; n < nchunks; ++n) {
         const int X = n & 1;
         uint8_t *stg = sm + (X ? OFF_REG1 : OFF_REG0);
         uint8_t *gro = sm + (X ? OFF_REG0 : OFF_REG1);
         const int t0 = n * CK;
-        const int nt = min(CK, T - t0);
 
-        // the previous chunk's O tile must have left X2 before this chunk writes there (after
-        // the barrier inside prep)
-        if (tid == 0) bulk_wait_read_all();
         if (!mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err)) break;
 
         // ============================================================ prep
-        if (tid < CK) BETAsm[tid] = beta_next;
-        beta_next = n + 1 < nchunks ? load_beta(n + 1) : 0.0f;
+        if (tid < CK) {
+            cp_async_wait_all();
+            const int t = t0 + tid;
+            const uint32_t wv = BRAW[(n & 1) * CK + tid];
+            const bool hi = t < T && (((uintptr_t)(p.beta + (size_t)(b * T + t) * p.H + h)) & 2);
+            BETAsm[tid] = __uint_as_float(hi ? (wv & 0xffff0000u) : (wv << 16));
+            if (n + 1 < nchunks) beta_async(n + 1);
+        }
         constexpr float INV_SC = 7.523164e-37f;    // SC = 2^120, INV_SC = 2^-120
         constexpr float LN_SC = 83.17766f;         // 120 ln 2
-        // pass 1: block log-decays L_B (sum of g over a 16-token block) per channel, and from
-        // them the per-(block, channel) factor table, computed once per chunk:
+        // pass 1, one (block, channel) per thread: block log-decay L_B (sum of g over the 16
+        // tokens), its first-half part H_B, and the factors
         //   fG = exp(G_blockstart)      fL = exp(G_C - G_blockend)
         //   fM = exp(-L_B / 2) / SC     (block-start reference, 1 / SC, where L_B < BAD_LOG)
-        //   fD = fM, or 0 where L_B < BAD_LOG (those diagonal terms are added exactly later)
-        //   fC(B, I) = exp(m_I - G_blockend of B) for later blocks I > B, m_I the reference of I
+        //   fC(B, I) = exp(m_I - G_blockend of B) for later blocks I > B, m_I the reference of I.
         // All exponents are sums of non-positive log-decays (plus L_B / 2 >= -84 for fM), so a
         // factor underflows only where the exact value does.
         {
-            const int c = tid >> 1, par = tid & 1;     // channel; blocks 2 par and 2 par + 1
+            const int c = tid >> 2, Bq = tid & 3;
             const uint8_t *gcol = stg + ST_G + (c >> 6) * 8192 + ((c & 7) << 1);
             const int chk = (c & 63) >> 3;
-            float Ls[2];
+            float h0 = 0.0f, h1 = 0.0f;
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float acc = 0.0f;
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    acc += __bfloat162float(*(const __nv_bfloat16 *)(gcol + swz(16 * (2 * par + u) + t, chk)));
-                Ls[u] = acc;
+            for (int t = 0; t < 16; ++t) {
+                // token order rotated by the block, so the four blocks' rows read by one warp
+                // instruction fall in different banks
+                const int tt = (t + 2 * Bq) & 15;
+                const float x = __bfloat162float(*(const __nv_bfloat16 *)(gcol + swz(16 * Bq + tt, chk)));
+                if (tt < 8) h0 += x;
+                else h1 += x;
             }
-            const float x0 = __shfl_xor_sync(0xffffffffu, Ls[0], 1), x1 = __shfl_xor_sync(0xffffffffu, Ls[1], 1);
-            const float Lv[4] = {par ? x0 : Ls[0], par ? x1 : Ls[1], par ? Ls[0] : x0, par ? Ls[1] : x1};
+            const float L = h0 + h1;
+            float Lv[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int Bq = 2 * par + u;
-                float lpre = 0.0f, lpost = 0.0f;
+            for (int J = 0; J < 4; ++J) Lv[J] = __shfl_sync(0xffffffffu, L, (lane & ~3) | J);
+            float lpre = 0.0f, lpost = 0.0f;
 #pragma unroll
-                for (int J = 0; J < 4; ++J) {
-                    if (J < Bq) lpre += Lv[J];
-                    if (J > Bq) lpost += Lv[J];
-                }
-                const bool badB = !(Ls[u] >= BAD_LOG);
-                const float fM = __expf((badB ? 0.0f : -0.5f * Ls[u]) - LN_SC);
-                FT[FT_G + Bq * DD + c] = __expf(lpre);
-                FT[FT_L + Bq * DD + c] = __expf(lpost);
-                FT[FT_M + Bq * DD + c] = fM;
-                FT[FT_D + Bq * DD + c] = badB ? 0.0f : fM;
-                if (badB) atomicOr(&badmask[Bq * 4 + (c >> 5)], 1u << (c & 31));
-#pragma unroll
-                for (int I = 1; I < 4; ++I) {
-                    if (I <= Bq) continue;
-                    float l = Lv[I] >= BAD_LOG ? 0.5f * Lv[I] : 0.0f;
-#pragma unroll
-                    for (int J = 1; J < 3; ++J)
-                        if (J > Bq && J < I) l += Lv[J];
-                    FT[FT_C + fc_slot(Bq, I) * DD + c] = __expf(l);
-                }
+            for (int J = 0; J < 4; ++J) {
+                if (J < Bq) lpre += Lv[J];
+                if (J > Bq) lpost += Lv[J];
             }
-            if (par == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
+            const bool badB = !(L >= BAD_LOG);
+            float *ft = FT + Bq * FSTRIDE + c;
+            ft[FT_G * FSTRIDE] = __expf(lpre);
+            ft[FT_L * FSTRIDE] = __expf(lpost);
+            ft[FT_M * FSTRIDE] = __expf((badB ? 0.0f : -0.5f * L) - LN_SC);
+            ft[FT_LB * FSTRIDE] = L;
+            ft[FT_H8 * FSTRIDE] = h0;
+            if (badB) atomicOr(&badmask[Bq * 4 + (c >> 5)], 1u << (c & 31));
+#pragma unroll
+            for (int I = 1; I < 4; ++I) {
+                if (I <= Bq) continue;
+                float l = Lv[I] >= BAD_LOG ? 0.5f * Lv[I] : 0.0f;
+#pragma unroll
+                for (int J = 1; J < 3; ++J)
+                    if (J > Bq && J < I) l += Lv[J];
+                FT[(FT_C + fc_slot(Bq, I)) * FSTRIDE + c] = __expf(l);
+            }
+            if (Bq == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
         }
         __syncthreads();
-        // pass 2: per token.  Lane (qq, a) of warp (B, cb) takes tokens 16 B + 4 qq + s, s < 4,
-        // and channels c0 .. c0 + 7.  With SC = 2^120:
+        // pass 2, per token.  Warp (pr, cq, th) takes token position p = lane & 7 of the half th
+        // of block pr (s = 0) and of block 3 - pr (s = 1), so every warp carries the same
+        // number of later-block Gram columns; lane >> 3 picks 8 of the 32 channels of quarter
+        // cq.  With SC = 2^120:
         //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
         //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
         // from log-domain prefix sums, so no partial product can underflow; both are normal
         // numbers for block log-decays down to BAD_LOG (SC e^-168 ~ e^-84.8).
         {
-            const int B = warp & 3;           // token block of this warp
-            const int cb = warp >> 2;         // channel block (64 channels)
-            const int qq = lane & 3;          // token quarter inside the block
-            const int a = lane >> 2;          // 16-byte chunk (8 channels) inside the channel block
+            const int pr = warp & 1;
+            const int cq = (warp >> 1) & 3;   // channel quarter (32 channels)
+            const int th = warp >> 3;         // token half of the block
+            const int pp = lane & 7;          // token position inside the half
+            const int a = 4 * (cq & 1) + (lane >> 3);   // 16-byte chunk inside the channel block
+            const int cb = cq >> 1;           // channel block (64 channels)
             const int c0 = 64 * cb + 8 * a;
-            float Gin[4][8], Lb[8];
-            {
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int i = 16 * B + 4 * qq + s;
-                    float gf[8];
-                    unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), gf);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) Gin[s][e] = (s == 0 ? 0.0f : Gin[s - 1][e]) + gf[e];
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    // exclusive prefix of the quarter log sums across the quad, and the block total
-                    float l = Gin[3][e];
-                    float y = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                    if (qq >= 1) l += y;
-                    y = __shfl_up_sync(0xffffffffu, l, 2, 4);
-                    if (qq >= 2) l += y;
-                    y = __shfl_up_sync(0xffffffffu, l, 1, 4);
-                    const float lex = qq >= 1 ? y : 0.0f;
-                    Lb[e] = __shfl_sync(0xffffffffu, l, (lane & ~3) | 3);
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) Gin[s][e] += lex;   // G_i - G_blockstart
-                }
-            }
-            auto ftab = [&](int off, float (&f)[8]) {
-                const float4 u0 = *(const float4 *)(FT + off + c0), u1 = *(const float4 *)(FT + off + c0 + 4);
+            auto ftab = [&](int row, float (&f)[8]) {
+                const float *src = FT + row * FSTRIDE + c0;
+                const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
                 f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
             };
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int i = 16 * B + 4 * qq + s;
+            for (int s = 0; s < 2; ++s) {
+                const int B = s == 0 ? pr : 3 - pr;
+                const int i = 16 * B + 8 * th + pp;
                 const uint32_t off = cb * 8192 + swz(i, a);
+                float Gin[8], Lb[8];
+                {
+                    // G_i - G_blockstart: inclusive scan over the 8 lanes of the half, plus H_B
+                    // for the second half
+                    float hb[8];
+                    ftab(FT_H8 + B, hb);
+                    unpack8(*(const uint4 *)(stg + ST_G + off), Gin);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float l = Gin[e];
+                        float y = __shfl_up_sync(0xffffffffu, l, 1, 8);
+                        if (pp >= 1) l += y;
+                        y = __shfl_up_sync(0xffffffffu, l, 2, 8);
+                        if (pp >= 2) l += y;
+                        y = __shfl_up_sync(0xffffffffu, l, 4, 8);
+                        if (pp >= 4) l += y;
+                        Gin[e] = l + (th ? hb[e] : 0.0f);
+                    }
+                    ftab(FT_LB + B, Lb);
+                }
+                const uint32_t badbits = (badmask[B * 4 + (c0 >> 5)] >> (c0 & 31)) & 0xffu;
                 float qf[8], kf[8], o[8], E1[8], E2[8], f[8];
                 unpack8(*(const uint4 *)(stg + ST_Q + off), qf);
                 unpack8(*(const uint4 *)(stg + ST_K + off), kf);
-                // exact diagonal of P: partial q_i . k_i over this lane's 8 channels
+                // exact diagonal of P: partial q_i . k_i over this lane's 8 channels, summed over
+                // the quarter's 4 lanes
                 float pd = 0.0f;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) pd += qf[e] * kf[e];
-                pd += __shfl_xor_sync(0xffffffffu, pd, 4);
                 pd += __shfl_xor_sync(0xffffffffu, pd, 8);
                 pd += __shfl_xor_sync(0xffffffffu, pd, 16);
-                if (a == 0) PDsm[cb * CK + i] = pd;
+                if (lane < 8) PDsm[cq * CK + i] = pd;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    E1[e] = __expf(Gin[s][e] + LN_SC);
-                    E2[e] = __expf(Lb[e] - Gin[s][e] + LN_SC);
+                    E1[e] = __expf(Gin[e] + LN_SC);
+                    E2[e] = __expf(Lb[e] - Gin[e] + LN_SC);
                 }
-                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA), Gamma_i = (E1 / SC) fG;
-                // odd quarters write their two 16-byte halves in the other order, which spreads
-                // each store over all 32 banks
-                ftab(FT_G + B * DD, f);
+                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA), Gamma_i = (E1 / SC) fG
+                ftab(FT_G + B, f);
                 float gam[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -365,24 +391,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 {
                     uint8_t *qh = sm + OFF_QH + (2 * cb + (a >> 2)) * 8192;
-                    const bool sw = qq & 1;
-                    const float4 lo4 = make_float4(o[0], o[1], o[2], o[3]), hi4 = make_float4(o[4], o[5], o[6], o[7]);
-                    *(float4 *)(qh + swz(i, 2 * (a & 3) + (sw ? 1 : 0))) = sw ? hi4 : lo4;
-                    *(float4 *)(qh + swz(i, 2 * (a & 3) + (sw ? 0 : 1))) = sw ? lo4 : hi4;
+                    *(float4 *)(qh + swz(i, 2 * (a & 3))) = make_float4(o[0], o[1], o[2], o[3]);
+                    *(float4 *)(qh + swz(i, 2 * (a & 3) + 1)) = make_float4(o[4], o[5], o[6], o[7]);
                 }
                 // K^ = Gamma k (in place)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * gam[e];
                 *(uint4 *)(stg + ST_K + off) = pack8(o);
                 // K~ = exp(G_C - G_i) k (over g) = k (E2 / SC) fL
-                ftab(FT_L + B * DD, f);
+                ftab(FT_L + B, f);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
                 *(uint4 *)(stg + ST_G + off) = pack8(o);
                 // Gram rows [Q_B; K_B] scaled by E1 fM = exp(G_i - m_B): hi part to the Gram
                 // rows, bf16 residual to X2 (free until the readback)
-                ftab(FT_M + B * DD, f);
-                const int rq = 32 * B + 4 * qq + s;
+                ftab(FT_M + B, f);
+                const int rq = 32 * B + 8 * th + pp;
                 {
                     float rf[8], hf[8], lo[8];
 #pragma unroll
@@ -405,13 +429,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     *(uint4 *)(gro + GR_R + cb * R_CB + swz(rq + 16, a)) = hk;
                     *(uint4 *)(sm + OFF_X2 + cb * R_CB + swz(rq + 16, a)) = pack8(lo);
                 }
-                // Gram columns, diagonal block: k E2 fD = k exp(m_B - G_j) (0 where L_B < BAD_LOG);
-                // hi part to diagonal column row i, bf16 residual over the (now dead) raw q
-                ftab(FT_D + B * DD, f);
+                // Gram columns, diagonal block: k E2 fM = k exp(m_B - G_j), 0 for channels with
+                // L_B < BAD_LOG (those terms are added exactly after the readback); hi part to
+                // diagonal column row i, bf16 residual over the (now dead) raw q
                 {
                     float hf[8], lo[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = kf[e] * (E2[e] * f[e]);
+                    for (int e = 0; e < 8; ++e) o[e] = (badbits >> e & 1u) ? 0.0f : kf[e] * (E2[e] * f[e]);
                     const uint4 hc = pack8(o);
                     unpack8(hc, hf);
 #pragma unroll
@@ -423,7 +447,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int I = 1; I < 4; ++I) {
                     if (I <= B) continue;
-                    ftab(FT_C + fc_slot(B, I) * DD, f);
+                    ftab(FT_C + fc_slot(B, I), f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
                     *(uint4 *)(gro + GR_CV + cb * CV_CB + swz(cv_off(I) + i, a)) = pack8(o);
@@ -434,7 +458,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tc_fence_before();
         __syncthreads();
 
-        // ============================================================ Gram + O init (MMA), decay S
+        // ============================================================ Gram (MMA)
         if (tid == 0) {
             tc_fence_after();
             const uint32_t sR = smem_u32(gro + GR_R), sCV = smem_u32(gro + GR_CV);
@@ -449,30 +473,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int kk = 0; kk < 8; ++kk)
                 mma_ss(tmem + TM_CORR, sdesc(sR + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
                        sdesc(sCVL + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_corr, 1);
-            // O^T = S^T Q^^T at tf32: A = fp32 state in TMEM, 8 key channels per MMA
-            const uint32_t sQ = smem_u32(sm + OFF_QH);
-            for (int kk = 0; kk < 16; ++kk)
-                mma_ts_tf32(tmem + TM_O, tmem + TM_S + kk * 8, sdesc(sQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                            id_o0, kk > 0);
             mma_commit(bar_mma);
         }
         if (!mma_wait()) break;
         tc_fence_after();
-        if (tid == 0 && n + 1 < nchunks) issue_tma(n + 1);   // the Gram region is free now
+        if (tid == 0 && n + 1 < nchunks) {
+            // the Gram region is free now; it was the stage of chunk n - 1, whose O tile must
+            // have been read out by its TMA store
+            bulk_wait_read_all();
+            issue_tma(n + 1);
+        }
 
         // ============================================================ Gram readback -> P, A
         {
-            const int I = warp & 3;
+            // lanes 0..15 of lane quarter I: P rows (q side), lanes 16..31: A rows (k side).
+            // CV_I has 2 (I + 1) chunks of 8 columns; chunk m goes to column group m % 4.
+            const int I = lq;
             const bool is_q = lane < 16;
             const int i = 16 * I + (lane & 15);
-            const int ncol = 8 * (I + 1);                 // this warp's share of CV_I
-            const int jbase = half * ncol;
+            const int nch = 2 * (I + 1);
             const float bi = BETAsm[i];
-            const float pdiag = PDsm[i] + PDsm[CK + i];   // exact q_i . k_i
-            const uint32_t *bmask = badmask + 4 * I;
-            // the warp's TMEM loads go out in two batches (earlier-block columns, then the
-            // diagonal block with its residual), one wait each; chunks are counted from the
-            // warp's last 8 columns, so only mm = 0, 1 can be diagonal
+            const float pdiag = (PDsm[i] + PDsm[CK + i]) + (PDsm[2 * CK + i] + PDsm[3 * CK + i]);   // exact q_i . k_i
             auto emit = [&](int j0, const uint32_t (&r)[8]) {
                 float vals[8];
 #pragma unroll
@@ -489,176 +510,179 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     unpack8(hi, hf);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) lo[e] = vals[e] - hf[e];
-                    *(uint4 *)(sm + OFF_P + swz(i, j0 >> 3)) = hi;
-                    *(uint4 *)(sm + OFF_PL + swz(i, j0 >> 3)) = pack8(lo);
+                    *(uint4 *)(stg + ST_P + swz(i, j0 >> 3)) = hi;
+                    *(uint4 *)(stg + ST_PL + swz(i, j0 >> 3)) = pack8(lo);
                 } else {
-                    *(float4 *)(A32 + i * 64 + j0) = make_float4(vals[0], vals[1], vals[2], vals[3]);
-                    *(float4 *)(A32 + i * 64 + j0 + 4) = make_float4(vals[4], vals[5], vals[6], vals[7]);
+                    *(float4 *)(A32 + aidx(i, j0)) = make_float4(vals[0], vals[1], vals[2], vals[3]);
+                    *(float4 *)(A32 + aidx(i, j0 + 4)) = make_float4(vals[4], vals[5], vals[6], vals[7]);
                 }
             };
-            {
-                uint32_t r[4][8];
+            uint32_t r[2][8], c8[2][8];
 #pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const int j0 = jbase + 8 * (I - mm);
-                    if (mm <= I && j0 < 16 * I) tmem_ld8(tmem + lane_q + TM_G + cv_off(I) + j0, r[mm]);
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const int j0 = jbase + 8 * (I - mm);
-                    if (mm <= I && j0 < 16 * I) emit(j0, r[mm]);
+            for (int u = 0; u < 2; ++u) {
+                const int m = cg + 4 * u;
+                if (m < 2 * I) {
+                    tmem_ld8(tmem + lane_q + TM_G + cv_off(I) + 8 * m, r[u]);   // earlier blocks
+                } else if (m < nch) {
+                    tmem_ld8(tmem + lane_q + TM_G + 8 * m, r[u]);               // own (diagonal) block
+                    tmem_ld8(tmem + lane_q + TM_CORR + 8 * m, c8[u]);
                 }
             }
-            {
-                uint32_t r[2][8], c8[2][8];
+            tmem_wait_ld();
 #pragma unroll
-                for (int mm = 0; mm < 2; ++mm) {
-                    const int j0 = jbase + 8 * (I - mm);
-                    if (mm <= I && j0 >= 16 * I) {
-                        tmem_ld8(tmem + lane_q + TM_G + j0, r[mm]);
-                        tmem_ld8(tmem + lane_q + TM_CORR + j0, c8[mm]);
-                    }
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int mm = 0; mm < 2; ++mm) {
-                    const int j0 = jbase + 8 * (I - mm);
-                    if (mm <= I && j0 >= 16 * I) {
+            for (int u = 0; u < 2; ++u) {
+                const int m = cg + 4 * u;
+                if (m < nch) {
+                    if (m >= 2 * I) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            r[mm][e] = __float_as_uint(__uint_as_float(r[mm][e]) + __uint_as_float(c8[mm][e]));
-                        emit(j0, r[mm]);
+                            r[u][e] = __float_as_uint(__uint_as_float(r[u][e]) + __uint_as_float(c8[u][e]));
                     }
+                    emit(8 * m, r[u]);
+                } else if (is_q) {
+                    // P is an MMA operand: its upper part must be zero (A's is never read)
+                    *(uint4 *)(stg + ST_P + swz(i, m)) = make_uint4(0, 0, 0, 0);
+                    *(uint4 *)(stg + ST_PL + swz(i, m)) = make_uint4(0, 0, 0, 0);
                 }
             }
             // exact diagonal-block terms of channels whose block decay underflows the Gram
             // factorisation, added in place to this thread's own entries (rare path)
+            const uint32_t *bmask = badmask + 4 * I;
             for (int wd = 0; wd < 4; ++wd) {
-                for (uint32_t m = bmask[wd]; m != 0u; m &= m - 1u) {
-                    const int c = 32 * wd + __ffs((int)m) - 1;
+                for (uint32_t mk = bmask[wd]; mk != 0u; mk &= mk - 1u) {
+                    const int c = 32 * wd + __ffs((int)mk) - 1;
                     const size_t rowi = ((size_t)(b * T + t0 + i) * p.H + h) * DD + c;
                     const float xi = (t0 + i < T) ? __bfloat162float((is_q ? p.q : p.k)[rowi]) : 0.0f;
                     float w = 1.0f;   // exp(G_i - G_j), built backwards from j = i
                     for (int j = i; j >= 16 * I; --j) {
                         const bool valid = t0 + j < T;
                         const size_t rowj = ((size_t)(b * T + t0 + j) * p.H + h) * DD + c;
-                        if (j < i && j >= jbase && j < jbase + ncol) {
+                        if (j < i && ((j >> 3) & 3) == cg) {
                             const float d = xi * (valid ? __bfloat162float(p.k[rowj]) : 0.0f) * w;
                             if (is_q) {
-                                __nv_bfloat16 *ph = (__nv_bfloat16 *)(sm + OFF_P + swz(i, j >> 3)) + (j & 7);
-                                __nv_bfloat16 *pl = (__nv_bfloat16 *)(sm + OFF_PL + swz(i, j >> 3)) + (j & 7);
+                                __nv_bfloat16 *ph = (__nv_bfloat16 *)(stg + ST_P + swz(i, j >> 3)) + (j & 7);
+                                __nv_bfloat16 *pl = (__nv_bfloat16 *)(stg + ST_PL + swz(i, j >> 3)) + (j & 7);
                                 const float v = __bfloat162float(*ph) + __bfloat162float(*pl) + d;
                                 const __nv_bfloat16 vh = __float2bfloat16_rn(v);
                                 *ph = vh;
                                 *pl = __float2bfloat16_rn(v - __bfloat162float(vh));
                             } else {
-                                A32[i * 64 + j] += bi * d;
+                                A32[aidx(i, j)] += bi * d;
                             }
                         }
                         w *= __expf(valid ? __bfloat162float(p.g[rowj]) : 0.0f);
                     }
                 }
             }
-            if (half == 1) {
-                for (int jc = 2 * (I + 1); jc < 8; ++jc) {
-                    if (is_q) {
-                        *(uint4 *)(sm + OFF_P + swz(i, jc)) = make_uint4(0, 0, 0, 0);
-                        *(uint4 *)(sm + OFF_PL + swz(i, jc)) = make_uint4(0, 0, 0, 0);
-                    } else {
-                        *(float4 *)(A32 + i * 64 + 8 * jc) = make_float4(0.f, 0.f, 0.f, 0.f);
-                        *(float4 *)(A32 + i * 64 + 8 * jc + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                }
-            }
         }
         __syncthreads();
         if (tid < 16) badmask[tid] = 0u;   // masks consumed
+        if (tid == NT - 32) {
+            // O^T = S^T Q^^T at tf32 (A = fp32 state in TMEM, 8 key channels per MMA), issued
+            // by the last warp, which has no part in the inverse; it runs while the CUDA cores
+            // invert, and completes on bar_o before the state is decayed
+            tc_fence_after();
+            const uint32_t sQ = smem_u32(sm + OFF_QH);
+            for (int kk = 0; kk < 16; ++kk)
+                mma_ts_tf32(tmem + TM_O, tmem + TM_S + kk * 8, sdesc(sQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                            id_o0, kk > 0);
+            mma_commit(bar_o);
+        }
 
         // ============================================================ T = (I + A)^{-1} Diag(beta)
-        // L = I + A, blocked by 16: diagonal inverses L_II^{-1} (right-looking forward
-        // substitution, one column per thread), then A''_IK = L_II^{-1} A_IK, then block rows
-        // by distance: T_IJ = -sum_{K=J}^{I-1} A''_IK T_KJ.  The block products run on
-        // strips of 4 rows x 1 column per thread (row segments read as float4).
+        // L = I + A, inverted in two levels of 2x2 blocks.  16x16 diagonal inverses L_II^{-1}
+        // by right-looking forward substitution (one column per thread); then each 32x32 half
+        //     [[L_a, 0], [A_ba, L_b]]^{-1} = [[L_a^{-1}, 0], [-L_b^{-1} A_ba L_a^{-1}, L_b^{-1}]]
+        // and the same rule once more for the 64x64 matrix with 32x32 blocks.  Every product
+        // is a full-precision fp32 dot product (16x16 blocks: one output per thread; 32x32
+        // blocks: 4 rows x 1 column per thread).  Scratch (P, Q) lives in A's unused
+        // upper-right 32x32 block.
         if (tid < 64) {
             const int Ib = tid >> 4, col = tid & 15;
-            const float *Ab = A32 + (16 * Ib) * 64 + 16 * Ib;
             float x[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.0f : 0.0f;
 #pragma unroll
             for (int m = 0; m < 15; ++m)
 #pragma unroll
-                for (int r = m + 1; r < 16; ++r) x[r] -= Ab[r * 64 + m] * x[m];
+                for (int r = m + 1; r < 16; ++r) x[r] -= A32[aidx(16 * Ib + r, 16 * Ib + m)] * x[m];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) LINV[(16 * Ib + r) * 64 + 16 * Ib + col] = x[r];
+            for (int r = 0; r < 16; ++r) LINV[aidx(16 * Ib + r, 16 * Ib + col)] = x[r];
         }
         __syncthreads();
-        {
-            const int set = tid >> 6;               // which block product this thread serves
-            const int r0 = ((tid >> 4) & 3) * 4;    // rows r0..r0+3 of the 16x16 block
-            const int cc = tid & 15;                // column
-            // acc[q] += sum_m X[rowbase + r0 + q][colX + m] * Y[rowY + m][colY + cc]
-            auto strip = [&](const float *X, int xrow, int xcol, const float *Y, int yrow, int ycol,
-                             float (&acc)[4]) {
+        // dot16(X, xr, xc, Y, yr, yc): sum_m X[xr][xc + m] Y[yr + m][yc], m < 16
+        auto dot16 = [&](const float *Xm, int xr, int xc, const float *Ym, int yr, int yc) -> float {
+            float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
-                for (int m4 = 0; m4 < 16; m4 += 4) {
-                    const float y0 = Y[(yrow + m4 + 0) * 64 + ycol + cc], y1 = Y[(yrow + m4 + 1) * 64 + ycol + cc];
-                    const float y2 = Y[(yrow + m4 + 2) * 64 + ycol + cc], y3 = Y[(yrow + m4 + 3) * 64 + ycol + cc];
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 xv = *(const float4 *)(Xm + aidx(xr, xc + m4));
+                s0 += xv.x * Ym[aidx(yr + m4 + 0, yc)] + xv.z * Ym[aidx(yr + m4 + 2, yc)];
+                s1 += xv.y * Ym[aidx(yr + m4 + 1, yc)] + xv.w * Ym[aidx(yr + m4 + 3, yc)];
+            }
+            return s0 + s1;
+        };
+        {
+            // 32x32 halves h = 0 (blocks 0, 1) and h = 1 (blocks 2, 3):
+            // P_h = A_{2h+1,2h} L_{2h}^{-1}  ->  scratch rows 0..15, columns 32 + 16 h ..
+            const int hh = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+            const int ra = 32 * hh, rb = 32 * hh + 16;
+            A32[aidx(r, 32 + 16 * hh + c)] = dot16(A32, rb + r, ra, LINV, ra, ra + c);
+            __syncthreads();
+            // T_{2h+1,2h} = -L_{2h+1}^{-1} P_h; the (2h, 2h+1) block is zero
+            LINV[aidx(rb + r, ra + c)] = -dot16(LINV, rb + r, rb, A32, 0, 32 + 16 * hh + c);
+            LINV[aidx(ra + r, rb + c)] = 0.0f;
+            __syncthreads();
+        }
+        {
+            // Q = A_{[2,3],[0,1]} L_{[0,1]}^{-1}: 4 rows x 1 column per thread (256 threads)
+            const int c = tid & 31, rg = (tid >> 5) & 7;   // rows 4 rg .. 4 rg + 3 of 32
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (tid < 256) {
+#pragma unroll
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    float y[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) y[t] = LINV[aidx(m4 + t, c)];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const float4 xv = *(const float4 *)(X + (xrow + r0 + q) * 64 + xcol + m4);
-                        acc[q] += xv.x * y0 + xv.y * y1 + xv.z * y2 + xv.w * y3;
+                        const float4 xv = *(const float4 *)(A32 + aidx(32 + 4 * rg + q, m4));
+                        acc[q] += xv.x * y[0] + xv.y * y[1] + xv.z * y[2] + xv.w * y[3];
                     }
                 }
-            };
-            // A''_IK for the 6 pairs (I, K), K < I: sets 0..3 take pairs {set, set + 4}
-            float y[2][4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int pi = set + 4 * u;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) y[u][q] = 0.0f;
-                if (pi < 6) {
-                    const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
-                    const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
-                    strip(LINV, 16 * I, 16 * I, A32, 16 * I, 16 * K, y[u]);
-                }
+                for (int q = 0; q < 4; ++q) A32[aidx(4 * rg + q, 32 + c)] = acc[q];
             }
             __syncthreads();
+            // T_{[2,3],[0,1]} = -L_{[2,3]}^{-1} Q
+            if (tid < 256) {
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int pi = set + 4 * u;
-                if (pi < 6) {
-                    const int I = pi < 1 ? 1 : (pi < 3 ? 2 : 3);
-                    const int K = pi < 1 ? 0 : (pi < 3 ? pi - 1 : pi - 3);
+                for (int q = 0; q < 4; ++q) acc[q] = 0.0f;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) A32[(16 * I + r0 + q) * 64 + 16 * K + cc] = y[u][q];
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    float y[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) y[t] = A32[aidx(m4 + t, 32 + c)];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 xv = *(const float4 *)(LINV + aidx(32 + 4 * rg + q, 32 + m4));
+                        acc[q] += xv.x * y[0] + xv.y * y[1] + xv.z * y[2] + xv.w * y[3];
+                    }
                 }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) LINV[aidx(32 + 4 * rg + q, c)] = -acc[q];
             }
             __syncthreads();
-#pragma unroll
-            for (int d = 1; d < 4; ++d) {
-                const int J = set, I = set + d;
-                if (I < 4) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int K = 0; K < 3; ++K)
-                        if (K >= J && K < I) strip(A32, 16 * I, 16 * K, LINV, 16 * K, 16 * J, acc);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) LINV[(16 * I + r0 + q) * 64 + 16 * J + cc] = -acc[q];
-                }
-                __syncthreads();
-            }
         }
-        for (int idx = tid; idx < 64 * 8; idx += NT) {
-            const int i = idx >> 3, jc = idx & 7;
+        {
+            // T = L^{-1} Diag(beta), lower triangle, bf16 K-major [i][j]
+            const int i = tid >> 3, jc = tid & 7;
+            const float4 l0 = *(const float4 *)(LINV + aidx(i, 8 * jc)), l1 = *(const float4 *)(LINV + aidx(i, 8 * jc + 4));
+            const float4 b0 = *(const float4 *)(BETAsm + 8 * jc), b1 = *(const float4 *)(BETAsm + 8 * jc + 4);
+            const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
             float vals[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int j = 8 * jc + e;
-                vals[e] = j <= i ? LINV[i * 64 + j] * BETAsm[j] : 0.0f;
-            }
+            for (int e = 0; e < 8; ++e) vals[e] = 8 * jc + e <= i ? lv[e] * bv[e] : 0.0f;
             *(uint4 *)(sm + OFF_T + swz(i, jc)) = pack8(vals);
         }
         fence_proxy_async();
@@ -678,15 +702,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mma_wait()) break;
         tc_fence_after();
         {
-            // W^T (lane = key channel c = 32 (warp & 3) + lane) -> W in shared memory, fp32 K-major [i][c]
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_q + TM_W + 32 * half, r);
+            // W^T (lane = key channel c = 32 lq + lane) -> W in shared memory, fp32 K-major [i][c];
+            // K-block c / 32 = this warp's lane quarter; one 128-byte row per token i
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_q + TM_W + 16 * cg, r);
             tmem_wait_ld();
-            // K-block c / 32 = this warp's lane quarter; a warp writes one 128-byte row per token i
-            uint8_t *wb = sm + OFF_W + (warp & 3) * 8192 + (lane & 3) * 4;
+            uint8_t *wb = sm + OFF_W + lq * 8192 + (lane & 3) * 4;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                *(uint32_t *)(wb + swz(32 * half + e, lane >> 2)) = r[e];
+            for (int e = 0; e < 16; ++e)
+                *(uint32_t *)(wb + swz(16 * cg + e, lane >> 2)) = r[e];
         }
         fence_proxy_async();
         tc_fence_before();
@@ -701,41 +725,38 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mma_commit(bar_mma);
         }
         if (!mma_wait()) break;
+        if (!mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err)) break;
         tc_fence_after();
         {
-            // U^T fp32 -> bf16 hi and lo A operands
-            uint32_t r[32], r8[8], l8[8];
-            tmem_ld32(tmem + lane_q + TM_U + 32 * half, r);
+            // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column)
+            uint32_t r[16], r8[8], l8[8];
+            tmem_ld16(tmem + lane_q + TM_U + 16 * cg, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x0 = __uint_as_float(r[16 * m + 2 * e]), x1 = __uint_as_float(r[16 * m + 2 * e + 1]);
-                    r8[e] = pack_bf16x2(x0, x1);
-                    const float2 hv = unpack_bf16x2(r8[e]);
-                    l8[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
-                }
-                tmem_st8(tmem + lane_q + TM_UB + 16 * half + 8 * m, r8);
-                tmem_st8(tmem + lane_q + TM_UL + 16 * half + 8 * m, l8);
+            for (int e = 0; e < 8; ++e) {
+                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                r8[e] = pack_bf16x2(x0, x1);
+                const float2 hv = unpack_bf16x2(r8[e]);
+                l8[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
             }
-            // S^T <- S^T Diag(exp G_C) (every reader of the chunk-start state has finished)
-            for (int cc = 0; cc < 64; cc += 32) {
-                const uint32_t ta = tmem + lane_q + TM_S + 64 * half + cc;
-                tmem_ld32(ta, r);
-                tmem_wait_ld();
+            tmem_st8(tmem + lane_q + TM_UB + 8 * cg, r8);
+            tmem_st8(tmem + lane_q + TM_UL + 8 * cg, l8);
+            // S^T <- S^T Diag(exp G_C) (every reader of the chunk-start state has finished: the
+            // O init was waited for above)
+            uint32_t sr[32];
+            const uint32_t ta = tmem + lane_q + TM_S + 32 * cg;
+            tmem_ld32(ta, sr);
+            tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    r[e] = __float_as_uint(__uint_as_float(r[e]) * GCsm[64 * half + cc + e]);
-                tmem_st32(ta, r);
-            }
+            for (int e = 0; e < 32; ++e) sr[e] = __float_as_uint(__uint_as_float(sr[e]) * GCsm[32 * cg + e]);
+            tmem_st32(ta, sr);
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t sP = smem_u32(sm + OFF_P), sPL = smem_u32(sm + OFF_PL), sG = smem_u32(stg + ST_G);
+            const uint32_t sP = smem_u32(stg + ST_P), sPL = smem_u32(stg + ST_PL), sG = smem_u32(stg + ST_G);
             for (int kk = 0; kk < 4; ++kk) {
                 mma_ts(tmem + TM_O, tmem + TM_UB + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
                 mma_ts(tmem + TM_O, tmem + TM_UL + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
@@ -750,23 +771,25 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!mma_wait()) break;
         tc_fence_after();
         {
-            // O^T -> bf16 tile in X2 (the load tiles' layout: 2 channel blocks of [64 rows x 128 B],
-            // 128-byte swizzle), then two TMA stores; rows past T are clipped by the tensor map
-            const int v = 32 * (warp & 3) + lane;
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_q + TM_O + 32 * half, r);
+            // O^T -> bf16 tile in the stage's V tile (dead since the U~ MMA; the load tiles'
+            // layout: 2 channel blocks of [64 rows x 128 B], 128-byte swizzle), then two TMA
+            // stores; rows past T are clipped by the tensor map.  The stores are waited for
+            // (read side) only before the next TMA load into this stage region.
+            const int v = 32 * lq + lane;
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_q + TM_O + 16 * cg, r);
             tmem_wait_ld();
-            uint8_t *ot = sm + OFF_X2 + (v >> 6) * 8192 + ((v & 7) << 1);
+            uint8_t *ot = stg + ST_V + (v >> 6) * 8192 + ((v & 7) << 1);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                *(__nv_bfloat16 *)(ot + swz(32 * half + e, (v & 63) >> 3)) = __float2bfloat16_rn(__uint_as_float(r[e]));
+            for (int e = 0; e < 16; ++e)
+                *(__nv_bfloat16 *)(ot + swz(16 * cg + e, (v & 63) >> 3)) = __float2bfloat16_rn(__uint_as_float(r[e]));
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            tma_store_4d(&tm_o, sm + OFF_X2, 0, h, t0, b);
-            tma_store_4d(&tm_o, sm + OFF_X2 + 8192, 64, h, t0, b);
+            tma_store_4d(&tm_o, stg + ST_V, 0, h, t0, b);
+            tma_store_4d(&tm_o, stg + ST_V + 8192, 64, h, t0, b);
             bulk_commit();
         }
     }
@@ -774,15 +797,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ---------------------------------------------------------------- final state
     if (p.sT && !*abort_flag) {
         tc_fence_after();
-        const int v = 32 * (warp & 3) + lane;
+        const int v = 32 * lq + lane;
         float *sT = p.sT + (size_t)bh * DD * DD;
-        for (int cc = 0; cc < 64; cc += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_q + TM_S + 64 * half + cc, r);
-            tmem_wait_ld();
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_q + TM_S + 32 * cg, r);
+        tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sT[(size_t)(64 * half + cc + e) * DD + v] = __uint_as_float(r[e]);
-        }
+        for (int e = 0; e < 32; ++e) sT[(size_t)(32 * cg + e) * DD + v] = __uint_as_float(r[e]);
     }
     if (tid == 0) bulk_wait_all();
     tc_fence_before();
@@ -844,8 +865,9 @@ bool device_is_sm100()
 
 bool chunk_tc_supported(const ChunkArgs &a)
 {
+    // beta is fetched as aligned 32-bit words (cp.async), so it must start on a 4-byte boundary
     return a.io == IO_BF16 && a.dk == DD && a.dv == DD && !a.qkv_f32 && !a.g_f32 && !a.beta_f32 && !a.out_f32 &&
-           a.T > 0 && device_is_sm100() && encode_fn() != nullptr;
+           a.T > 0 && ((uintptr_t)a.beta & 3) == 0 && device_is_sm100() && encode_fn() != nullptr;
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)

@@ -66,6 +66,16 @@ KDA_DEVICE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *
     }
 }
 
+// ------------------------------------------------------------------ cp.async (4 bytes)
+// Global -> shared copy of one aligned 32-bit word without a register: src_bytes (0, 2 or 4)
+// are read from src, the rest of the word is zero-filled.  src must be 4-byte aligned.
+KDA_DEVICE void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+KDA_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+KDA_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA
 // 4-D tiled load into shared memory, completing on `bar` (transaction bytes).
 KDA_DEVICE void tma_load_4d(void *smem_dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
@@ -126,6 +136,14 @@ KDA_DEVICE void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7])
+                 : "r"(taddr));
+}
+KDA_DEVICE void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15])
                  : "r"(taddr));
 }
 KDA_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
