@@ -112,6 +112,7 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
     kda::ChunkArgs a{q, k, v, g, beta, initial_state, out, final_state, B, T, H, dk, dv,
                      io_of(io), false, false, false, false, error_word()};
     if (kda::chunk_tc_supported(a)) return cuda_status(kda::launch_chunk_tc(a, s));
+    if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
     return cuda_status(kda::launch_chunk_simt(a, s));
 }
 
@@ -174,7 +175,7 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     kda::ChunkArgs ca{wq, wk, wv, wg, wb, initial_state, wo, final_state, B, T, H, dk, dv,
                       kda::IO_F32, true, true, true, true, error_word()};
-    e = kda::launch_chunk_simt(ca, s);
+    e = kda::chunk_f32_supported(ca) ? kda::launch_chunk_f32(ca, s) : kda::launch_chunk_simt(ca, s);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     kda::EpilogueArgs ea{wo, o_gate_raw, o_norm_w, norm_eps, out, B, T, H, dv, io_of(io)};
     return cuda_status(kda::launch_epilogue(ea, s));

@@ -51,6 +51,9 @@ struct EpilogueArgs {
 
 // CUDA-core chunked kernel: any supported dtype, dk, dv in {64, 128}.
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
+// Exact fp32 chunked kernel on CUDA cores for dk = dv = 128 with all-fp32 operands.
+cudaError_t launch_chunk_f32(const ChunkArgs &a, cudaStream_t s);
+bool chunk_f32_supported(const ChunkArgs &a);
 // tcgen05 chunked kernel: bf16 I/O, dk = dv = 128.
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 bool chunk_tc_supported(const ChunkArgs &a);

@@ -46,9 +46,12 @@ BF16_FORMAT_REL = 2.0 ** -8
 
 
 def err(gpu, ref, io, stored_bf16=None):
-    """Error as a fraction of the allowed bound (passes when <= 1).  `stored_bf16` says
-    whether the GPU value was stored in bf16 (outputs under bf16 I/O); the final state is
-    always fp32."""
+    """Error as a fraction of the allowed bound (passes when <= 1).  `stored_bf16` is the
+    number of bf16 roundings the GPU value went through (True = 1: outputs under bf16 I/O;
+    2: the layer output, whose RMSNorm casts to the activation dtype before the gain and
+    gate and the result is stored in bf16 again; 0 / False: the fp32 final state).  Each
+    rounding of a value that differs from the oracle's by any amount may land one bf16 step
+    (2^-8 relative) apart."""
     gpu, ref = np.asarray(gpu, np.float64), np.asarray(ref, np.float64)
     assert np.all(np.isfinite(gpu)), "non-finite GPU output"
     if gpu.size == 0:
@@ -60,7 +63,7 @@ def err(gpu, ref, io, stored_bf16=None):
         stored_bf16 = True
     bound = TOL_BF16 * max(np.sqrt(np.mean(ref * ref)), 1e-30)
     if stored_bf16:
-        bound = bound + BF16_FORMAT_REL * np.abs(ref)
+        bound = bound + int(stored_bf16) * BF16_FORMAT_REL * np.abs(ref)
     return float(np.max(d / bound))
 
 
@@ -99,10 +102,10 @@ def oracle_prefill(d, heads=None):
                             np.ascontiguousarray(beta[bs, :, hs].T[None]), s0s)
 
 
-def check_heads(out, sT, ref_o, ref_s, heads, io):
+def check_heads(out, sT, ref_o, ref_s, heads, io, roundings=1):
     o_gpu = np.stack([f64(out[b, :, h]) for b, h in heads], axis=1)[None]
     s_gpu = np.stack([f64(sT[b, h]) for b, h in heads], axis=0)[None]
-    eo, es = err(o_gpu, ref_o, io), serr(s_gpu, ref_s, io)
+    eo, es = err(o_gpu, ref_o, io, stored_bf16=roundings), serr(s_gpu, ref_s, io)
     assert eo <= 1.0, f"output error {eo:.3e} of bound"
     assert es <= 1.0, f"state error {es:.3e} of bound"
     return eo, es
@@ -199,29 +202,37 @@ def test_state_passing_in_place_across_calls(kda, io):
     assert serr(f64(S), rs, io) <= 1.0
 
 
-@pytest.mark.parametrize("gval", [-40.0, -1e-4])
-def test_extreme_gates(kda, gval):
-    """Very strong (-40 per step) and very weak (-1e-4 per step) decay on every channel."""
-    d = inputs.prefill_inputs(1, 200, 2, 128, 128, io="bf16", seed=8, s0_std=0.05)
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("gval", [-40.0, -9.0, -1e-4])
+def test_extreme_gates(kda, io, gval):
+    """Very strong (-40 per step: every block's decay below e^-168, the exact diagonal
+    path on every channel), strong (-9: the fp32 kernel's exact path, not the tensor-core
+    kernel's) and very weak (-1e-4 per step) decay on every channel."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(1, 200, 2, 128, 128, io=ioname, seed=8, s0_std=0.05)
     d["g"] = torch.full_like(d["g"], gval)
     out, sT = run_prefill(kda, d)
     ro, rs = oracle_prefill(d)
-    assert err(f64(out), ro, torch.bfloat16) <= 1.0
-    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+    assert err(f64(out), ro, io) <= 1.0
+    assert serr(f64(sT), rs, io) <= 1.0
 
 
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("bval", [0.0, 1.0])
-def test_beta_extremes(kda, bval):
-    d = inputs.prefill_inputs(1, 150, 2, 128, 128, io="bf16", seed=9, s0_std=0.05)
+def test_beta_extremes(kda, io, bval):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(1, 150, 2, 128, 128, io=ioname, seed=9, s0_std=0.05)
     d["beta"] = torch.full_like(d["beta"], bval)
     out, sT = run_prefill(kda, d)
     ro, rs = oracle_prefill(d)
-    assert err(f64(out), ro, torch.bfloat16) <= 1.0
-    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+    assert err(f64(out), ro, io) <= 1.0
+    assert serr(f64(sT), rs, io) <= 1.0
 
 
-def test_prefill_is_deterministic(kda):
-    d = inputs.prefill_inputs(2, 300, 4, 128, 128, io="bf16", seed=10, s0_std=0.02)
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_prefill_is_deterministic(kda, io):
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.prefill_inputs(2, 300, 4, 128, 128, io=ioname, seed=10, s0_std=0.02)
     o1, s1 = run_prefill(kda, d)
     o2, s2 = run_prefill(kda, d)
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
@@ -336,7 +347,7 @@ def test_layer_small(kda, io, d_, T):
                             dt_bias_std=0.5, gain_std=0.2)
     out, sT = run_layer(kda, d)
     ro, rs = oracle_layer(d, io)
-    assert err(f64(out), ro, io) <= tol(io)
+    assert err(f64(out), ro, io, stored_bf16=2) <= tol(io)
     assert serr(f64(sT), rs, io) <= 1.0
 
 
@@ -348,7 +359,7 @@ def test_layer_workload_B2_T16384_H96_sampled_heads(kda):
     out, sT = run_layer(kda, d)
     heads = [(0, 0), (1, 95), (0, 50), (1, 13)]
     ro, rs = oracle_layer(d, torch.bfloat16, heads)
-    check_heads(out, sT, ro, rs, heads, torch.bfloat16)
+    check_heads(out, sT, ro, rs, heads, torch.bfloat16, roundings=2)
 
 
 def test_layer_zero_gate_input_halves_output(kda):
