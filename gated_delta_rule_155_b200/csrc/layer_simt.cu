@@ -1,6 +1,6 @@
 // layer_simt.cu — KDA layer prologue and epilogue as streaming CUDA-core kernels.
 //
-// Prologue, per (b, t, h) token-head (one warp each):
+// Prologue, per (b, h) and run of 8 tokens (one warp each):
 //   q = l2norm(SiLU(conv_q * q_raw)),  k = l2norm(SiLU(conv_k * k_raw)),  v = SiLU(conv_v * v_raw)
 //     depthwise causal conv of kernel 4 with zero history, PyTorch Conv1d tap order:
 //     y[t, c] = sum_{i=0..3} w[c, i] x[t - 3 + i, c]
@@ -24,21 +24,75 @@ namespace {
 constexpr int LY_THREADS = 256;
 constexpr float L2_EPS = 1e-6f;
 
-template <typename IO, int D>
-KDA_DEVICE void conv_row(const IO *__restrict__ x, const float *__restrict__ w, int t, size_t row_stride,
-                         int c0, float (&y)[D / 32])
+constexpr int RUN = 8;   // tokens per warp in the prologue
+
+// N consecutive elements (N = 2 or 4) as floats, and N floats stored
+template <int N> KDA_DEVICE void ldn(const float *p, float (&o)[N])
 {
-    // x points at (b, t=0, channel h*D); lane handles channels c0 + 32*e
+    if constexpr (N == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
+    } else {
+        const float2 t = *reinterpret_cast<const float2 *>(p);
+        o[0] = t.x; o[1] = t.y;
+    }
+}
+template <int N> KDA_DEVICE void ldn(const __nv_bfloat16 *p, float (&o)[N])
+{
+    if constexpr (N == 4) {
+        ld4(p, o);
+    } else {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+        o[0] = f.x; o[1] = f.y;
+    }
+}
+template <int N> KDA_DEVICE void stn(float *p, const float (&v)[N])
+{
+    if constexpr (N == 4) *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+}
+
+// One head's channels of one input stream over a run of tokens t0 .. t0 + nt - 1: causal
+// depthwise conv (PyTorch Conv1d tap order: y[t, c] = sum_i w[c, i] x[t - 3 + i, c], zero
+// history) + SiLU [+ L2-norm over the head's D channels].  Lane l owns channels
+// N l .. N l + N - 1 and slides a three-row window, so every input row is read once.
+template <typename IO, int D, bool NORM>
+KDA_DEVICE void conv_stream(const IO *__restrict__ x, size_t rs, const float *__restrict__ w, float *__restrict__ dst,
+                            size_t drs, int t0, int nt, int lane)
+{
+    constexpr int N = D / 32;
+    const int c0 = N * lane;
+    float wt[N][4], x3[N], x2[N], x1[N];
 #pragma unroll
-    for (int e = 0; e < D / 32; ++e) {
-        const int c = c0 + 32 * e;
-        const float4 wc = *reinterpret_cast<const float4 *>(w + (size_t)c * 4);
-        float acc = 0.0f;
-        if (t >= 3) acc += wc.x * to_f32(x[(size_t)(t - 3) * row_stride + c]);
-        if (t >= 2) acc += wc.y * to_f32(x[(size_t)(t - 2) * row_stride + c]);
-        if (t >= 1) acc += wc.z * to_f32(x[(size_t)(t - 1) * row_stride + c]);
-        acc += wc.w * to_f32(x[(size_t)t * row_stride + c]);
-        y[e] = siluf_(acc);
+    for (int e = 0; e < N; ++e) {
+        const float4 wv = *reinterpret_cast<const float4 *>(w + (size_t)(c0 + e) * 4);
+        wt[e][0] = wv.x; wt[e][1] = wv.y; wt[e][2] = wv.z; wt[e][3] = wv.w;
+        x3[e] = x2[e] = x1[e] = 0.0f;
+    }
+    if (t0 >= 3) ldn<N>(x + (size_t)(t0 - 3) * rs + c0, x3);
+    if (t0 >= 2) ldn<N>(x + (size_t)(t0 - 2) * rs + c0, x2);
+    if (t0 >= 1) ldn<N>(x + (size_t)(t0 - 1) * rs + c0, x1);
+    for (int r = 0; r < nt; ++r) {
+        const int t = t0 + r;
+        float xt[N], y[N];
+        ldn<N>(x + (size_t)t * rs + c0, xt);
+        float ss = 0.0f;
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+            float acc = wt[e][0] * x3[e];
+            acc += wt[e][1] * x2[e];
+            acc += wt[e][2] * x1[e];
+            acc += wt[e][3] * xt[e];
+            y[e] = siluf_(acc);
+            ss += y[e] * y[e];
+            x3[e] = x2[e]; x2[e] = x1[e]; x1[e] = xt[e];
+        }
+        if (NORM) {
+            const float sc = rsqrtf(warp_sum(ss) + L2_EPS);
+#pragma unroll
+            for (int e = 0; e < N; ++e) y[e] *= sc;
+        }
+        stn<N>(dst + (size_t)t * drs + c0, y);
     }
 }
 
@@ -46,55 +100,45 @@ template <typename IO, int DK, int DV>
 __global__ void __launch_bounds__(LY_THREADS)
 kda_prologue_kernel(PrologueArgs a)
 {
-    const int warp = (blockIdx.x * LY_THREADS + threadIdx.x) >> 5;
+    // one warp per (b, h, run of RUN tokens); consecutive warps take consecutive heads
+    const long long warp = ((long long)blockIdx.x * LY_THREADS + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    const long long ntok = (long long)a.B * a.T * a.H;
-    if (warp >= ntok) return;
-    const int h = warp % a.H;
-    const long long bt = warp / a.H;
-    const int t = (int)(bt % a.T);
-    const long long b = bt / a.T;
+    const int nrun = (a.T + RUN - 1) / RUN;
+    if (warp >= (long long)a.B * a.H * nrun) return;
+    const int h = (int)(warp % a.H);
+    const long long br = warp / a.H;
+    const int t0 = (int)(br % nrun) * RUN;
+    const int b = (int)(br / nrun);
+    const int nt = min(RUN, a.T - t0);
     const size_t rsk = (size_t)a.H * DK, rsv = (size_t)a.H * DV;
+    const size_t bt0 = (size_t)b * a.T;   // first (b, t) row of this sequence
 
-    // q, k: conv + SiLU + L2-norm over the head's dk channels
+    conv_stream<IO, DK, true>((const IO *)a.q_raw + bt0 * rsk + (size_t)h * DK, rsk, a.conv_q + (size_t)h * DK * 4,
+                              a.q + (bt0 * a.H + h) * DK, rsk, t0, nt, lane);
+    conv_stream<IO, DK, true>((const IO *)a.k_raw + bt0 * rsk + (size_t)h * DK, rsk, a.conv_k + (size_t)h * DK * 4,
+                              a.k + (bt0 * a.H + h) * DK, rsk, t0, nt, lane);
+    conv_stream<IO, DV, false>((const IO *)a.v_raw + bt0 * rsv + (size_t)h * DV, rsv, a.conv_v + (size_t)h * DV * 4,
+                               a.v + (bt0 * a.H + h) * DV, rsv, t0, nt, lane);
+    // gate g = -exp(A_log[h]) softplus(g_raw + dt_bias[h, c]) and beta = sigmoid(b_raw)
     {
-        const IO *xq = (const IO *)a.q_raw + (size_t)b * a.T * rsk + (size_t)h * DK;
-        const IO *xk = (const IO *)a.k_raw + (size_t)b * a.T * rsk + (size_t)h * DK;
-        float yq[DK / 32], yk[DK / 32];
-        conv_row<IO, DK>(xq, a.conv_q + (size_t)h * DK * 4, t, rsk, lane, yq);
-        conv_row<IO, DK>(xk, a.conv_k + (size_t)h * DK * 4, t, rsk, lane, yk);
-        float sq = 0.f, sk = 0.f;
-#pragma unroll
-        for (int e = 0; e < DK / 32; ++e) { sq += yq[e] * yq[e]; sk += yk[e] * yk[e]; }
-        sq = rsqrtf(warp_sum(sq) + L2_EPS);
-        sk = rsqrtf(warp_sum(sk) + L2_EPS);
-        const size_t o = (size_t)warp * DK;
-#pragma unroll
-        for (int e = 0; e < DK / 32; ++e) {
-            a.q[o + lane + 32 * e] = yq[e] * sq;
-            a.k[o + lane + 32 * e] = yk[e] * sk;
-        }
-    }
-    // v: conv + SiLU
-    {
-        const IO *xv = (const IO *)a.v_raw + (size_t)b * a.T * rsv + (size_t)h * DV;
-        float yv[DV / 32];
-        conv_row<IO, DV>(xv, a.conv_v + (size_t)h * DV * 4, t, rsv, lane, yv);
-        const size_t o = (size_t)warp * DV;
-#pragma unroll
-        for (int e = 0; e < DV / 32; ++e) a.v[o + lane + 32 * e] = yv[e];
-    }
-    // gate and beta
-    {
+        constexpr int N = DK / 32;
+        const int c0 = N * lane;
         const float scale = __expf(a.A_log[h]);
-        const IO *gr = (const IO *)a.g_raw + (size_t)warp * DK;
+        float bias[N];
 #pragma unroll
-        for (int e = 0; e < DK / 32; ++e) {
-            const int c = lane + 32 * e;
-            const float bias = a.dt_bias ? a.dt_bias[(size_t)h * DK + c] : 0.0f;
-            a.g[(size_t)warp * DK + c] = -scale * softplusf_(to_f32(gr[c]) + bias);
+        for (int e = 0; e < N; ++e) bias[e] = a.dt_bias ? a.dt_bias[(size_t)h * DK + c0 + e] : 0.0f;
+        for (int r = 0; r < nt; ++r) {
+            const size_t row = ((bt0 + t0 + r) * a.H + h) * DK + c0;
+            float x[N];
+            ldn<N>((const IO *)a.g_raw + row, x);
+#pragma unroll
+            for (int e = 0; e < N; ++e) x[e] = -scale * softplusf_(x[e] + bias[e]);
+            stn<N>(a.g + row, x);
         }
-        if (lane == 0) a.beta[warp] = sigmoidf_(to_f32(((const IO *)a.b_raw)[warp]));
+        if (lane < nt) {
+            const size_t th = (bt0 + t0 + lane) * a.H + h;
+            a.beta[th] = sigmoidf_(to_f32(((const IO *)a.b_raw)[th]));
+        }
     }
 }
 
@@ -132,7 +176,7 @@ __global__ void kda_fill_state_kernel(const float *__restrict__ s0, float *__res
 template <typename IO, int DK>
 cudaError_t launch_pro_dk(const PrologueArgs &a, cudaStream_t s)
 {
-    const long long warps = (long long)a.B * a.T * a.H;
+    const long long warps = (long long)a.B * a.H * ((a.T + RUN - 1) / RUN);
     const unsigned blocks = (unsigned)((warps * 32 + LY_THREADS - 1) / LY_THREADS);
     if (a.dv == 64) kda_prologue_kernel<IO, DK, 64><<<blocks, LY_THREADS, 0, s>>>(a);
     else kda_prologue_kernel<IO, DK, 128><<<blocks, LY_THREADS, 0, s>>>(a);
