@@ -2,22 +2,20 @@
 //
 // One CTA owns one (b, h) head and walks its chunks of C = 64 tokens in order.  The
 // fp32 state lives in tensor memory for the whole sequence, transposed (lane = value
-// column v, column = key channel c), next to its bf16 copy that feeds the MMAs as
-// the A operand.  Per chunk, with G_i = sum_{s<=i} g_s (per channel) and blocks of 16
-// tokens inside the chunk:
+// column v, column = key channel c).  Per chunk, with G_i = sum_{s<=i} g_s (per channel)
+// and blocks of 16 tokens inside the chunk:
 //
-//   prep (CUDA cores)   alpha = exp(g); in-block prefix/suffix products give
-//                       e1_i = exp(G_i - G_start(blk)), e2_i = exp(G_end(blk) - G_i) and the
-//                       block decays D_B; from them Q^ = Gamma*Q, K^ = Gamma*K,
-//                       K~ = exp(G_C - G)*K and the Gram operands (below).
+//   prep (CUDA cores)   per-(block, channel) decay factors, then Q^ = Gamma*Q (fp32),
+//                       K^ = Gamma*K, K~ = exp(G_C - G)*K and the Gram operands (below).
 //   Gram (tcgen05)      [Q;K] rows x CV_I columns -> P (j <= i) and A' (j < i) in one
-//                       M=128, N=160, K=128 MMA.
-//   inverse (CUDA)      T = (I + Diag(beta) A')^{-1} Diag(beta), blocked by 16, fp32.
-//   W, U~ (tcgen05)     W^T = K^^T T^T, U~^T = V^T T^T.
-//   chain (tcgen05)     U^T = U~^T - S^T W^T;  O^T = S^T Q^^T + U^T P^T;
-//                       S^T <- S^T Diag(exp G_C) + U^T K~.
-// The two products that read the state (S^T Q^^T and S^T W^T) run as kind::tf32 MMAs
-// with the fp32 state itself, straight from tensor memory, as the A operand.
+//                       M=128, N=160, K=128 MMA, plus a residual MMA for the diagonal blocks.
+//   inverse (CUDA)      T = (I + Diag(beta) A')^{-1} Diag(beta), blocked, fp32 — while the
+//                       tensor cores compute O^T = S^T Q^^T and Y^T = S^T K^^T.
+//   U (tcgen05)         U^T = V^T T^T - Y^T T^T, i.e. U = T (V - K^ S).
+//   chain (tcgen05)     O^T += U^T P^T;  S^T <- S^T Diag(exp G_C) + U^T K~.
+// The product that reads the state for the output (S^T Q^^T) runs as a kind::tf32 MMA with
+// the fp32 state itself as the TMEM A operand; Y = K^ S uses the state split into bf16
+// hi + lo parts.
 //
 // Overflow-safe Gram factorisation.  exp(G_i - G_j) (j <= i) spans far more than the
 // fp32 range over a chunk, so it is never formed as exp(G_i) exp(-G_j).  Row i of
@@ -33,9 +31,10 @@
 // Precision.  bf16 operands alone would put errors of the order of one bf16 rounding
 // on top of the output's own bf16 rounding.  So the diagonal P[i][i] = q_i . k_i is
 // formed exactly in fp32 from the raw inputs, the diagonal 16x16 blocks of the Gram get a
-// second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U and P enter their products as
-// hi + lo bf16 pairs (O += U_hi P_hi + U_lo P_hi + U_hi P_lo, S += K~^T (U_hi + U_lo)),
-// and the state is read at tf32 precision from its fp32 copy (Q^ and W kept in fp32).
+// second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U, Y and P enter their
+// products as hi + lo bf16 pairs (O += U_hi P_hi + U_lo P_hi + U_hi P_lo,
+// S += K~^T (U_hi + U_lo)), and the state is read at tf32 precision from its fp32 copy for
+// S^T Q^^T (Q^ kept in fp32).
 #include <cuda.h>
 
 #include <mutex>
@@ -64,10 +63,10 @@ constexpr int R_CB = 16384;                      // R: 128 rows x 128 B per chan
 constexpr int CV_ROWS = 160, CV_CB = CV_ROWS * 128;
 // X1 (32 KB): Q^ in fp32 (tf32 K-major [i][c]), from prep until the O-init MMA (issued
 // after the Gram readback) has run
-// X2 (32 KB): R_lo (prep -> Gram); A and L^{-1} in fp32 (inverse); W in fp32 (tf32 K-major
-// [i][c]); the O tile
+// X2 (32 KB): R_lo (prep -> Gram); then A and L^{-1} in fp32 (inverse)
 // P and P_lo (bf16 K-major [i][j], 8 KB each) take the stage's q tile once the Gram MMAs have
-// read the residual columns kept there; T (bf16 K-major [i][j], 8 KB) sits in the factor table
+// read the residual columns kept there; T (bf16 K-major [i][j], 8 KB) sits in the factor
+// table; the O tile is staged in the stage's V tile
 constexpr int OFF_X1 = 2 * REG_BYTES;
 constexpr int OFF_QH = OFF_X1;                   // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
 constexpr int ST_P = ST_Q, ST_PL = ST_Q + 8192;  // inside the stage region
@@ -78,7 +77,6 @@ constexpr int OFF_X2 = OFF_X1 + 32768;
 constexpr int AST = 68;
 constexpr int OFF_A32 = OFF_X2;
 constexpr int OFF_LINV = OFF_X2 + 64 * AST * 4;
-constexpr int OFF_W = OFF_X2;                    // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
 // per-(block, channel) table, fp32 rows of FSTRIDE (128 channels + padding that puts the
 // four blocks of one channel in different banks): fG, fL, fM, block log-decay L_B and
 // first-half log-decay H_B (tokens 0..7 of the block) for blocks 0..3, then fC for the six
@@ -93,9 +91,9 @@ constexpr int MS_BADMASK = 0;                    // uint32 [4][4]: channels with
 constexpr int MS_GC = 64;                        // fp32 [128] chunk decay exp(G_C)
 constexpr int MS_BETA = 576;                     // fp32 [64]
 constexpr int MS_PD = 832;                       // fp32 [4][64]: exact q_i . k_i, per channel quarter
-constexpr int MS_BAR = 1856;                     // uint64 [4]: tma0, tma1, mma, O init
-constexpr int MS_TSLOT = 1888;                   // uint32
-constexpr int MS_ABORT = 1892;                   // int
+constexpr int MS_BAR = 1856;                     // uint64 [5]: tma0, tma1, mma, O init, Y
+constexpr int MS_TSLOT = 1896;                   // uint32
+constexpr int MS_ABORT = 1900;                   // int
 constexpr int MS_BRAW = 1920;                    // uint32 [2][64]: beta words in flight (cp.async)
 constexpr int MISC_BYTES = 2432;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
@@ -106,14 +104,16 @@ __host__ __device__ constexpr int fc_slot(int B, int I) { return B == 0 ? I - 1 
 KDA_DEVICE int aidx(int i, int j) { return i * AST + j; }
 
 // tensor memory columns
-constexpr uint32_t TM_S = 0;     // fp32 S^T, 128 cols
-constexpr uint32_t TM_G = 128;   // Gram D, 160 cols (W^T reuses the first 64)
-constexpr uint32_t TM_W = 128;
-constexpr uint32_t TM_UL = 192;  // bf16 (U - U_hi)^T (A operand), 32 cols, inside the Gram area
-constexpr uint32_t TM_U = 288;   // U^T, 64 cols
-constexpr uint32_t TM_O = 352;   // O^T, 64 cols
+constexpr uint32_t TM_S = 0;       // fp32 S^T, 128 cols
+constexpr uint32_t TM_G = 128;     // Gram D, 160 cols; after the Gram readback:
+constexpr uint32_t TM_SH = 128;    //   bf16 S^T hi (A operand), 64 cols
+constexpr uint32_t TM_SL = 192;    //   bf16 S^T lo, 64 cols
+constexpr uint32_t TM_HI32 = 256;  //   bf16 Y^T hi, then U^T hi (A operands), 32 cols
+constexpr uint32_t TM_U = 288;     // U^T, 64 cols
+constexpr uint32_t TM_O = 352;     // O^T, 64 cols
 constexpr uint32_t TM_CORR = 416;  // diagonal-block Gram correction R_lo CVd + R CVd_lo, 64 cols
-constexpr uint32_t TM_UB = 480;  // bf16 U^T (A operand), 32 cols
+constexpr uint32_t TM_Y = 416;     //   then Y^T = S^T K^^T, 64 cols
+constexpr uint32_t TM_LO32 = 480;  // bf16 Y^T lo, then U^T lo, 32 cols
 
 // Gram column buffer: rows 0..63 are the diagonal-block columns (row j for token j);
 // rows cv_off(I) + j (j < 16 I) are block I's columns for earlier tokens.
@@ -156,6 +156,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *bar_tma = (uint64_t *)(misc + MS_BAR);
     uint64_t *bar_mma = bar_tma + 2;
     uint64_t *bar_o = bar_tma + 3;
+    uint64_t *bar_y = bar_tma + 4;
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
     float *A32 = (float *)(sm + OFF_A32);
@@ -175,6 +176,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&bar_tma[1], 1);
         mbar_init(bar_mma, 1);
         mbar_init(bar_o, 1);
+        mbar_init(bar_y, 1);
         *abort_flag = 0;
         for (int i = 0; i < 16; ++i) badmask[i] = 0u;
         fence_mbar_init();
@@ -227,7 +229,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr uint32_t id_corr = idesc_bf16(128, 64, false, false);
     constexpr uint32_t id_o0 = idesc_tf32(128, 64, false, false);
     constexpr uint32_t id_wt = idesc_bf16(128, 64, true, false);
-    constexpr uint32_t id_u = idesc_tf32(128, 64, false, false, true);
+    constexpr uint32_t id_opn = idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t id_op = idesc_bf16(128, 64, false, false);
     constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
 
@@ -577,67 +579,65 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         __syncthreads();
         if (tid < 16) badmask[tid] = 0u;   // masks consumed
-        if (tid == NT - 32) {
-            // O^T = S^T Q^^T at tf32 (A = fp32 state in TMEM, 8 key channels per MMA), issued
-            // by the last warp, which has no part in the inverse; it runs while the CUDA cores
-            // invert, and completes on bar_o before the state is decayed
-            tc_fence_after();
-            const uint32_t sQ = smem_u32(sm + OFF_QH);
-            for (int kk = 0; kk < 16; ++kk)
-                mma_ts_tf32(tmem + TM_O, tmem + TM_S + kk * 8, sdesc(sQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                            id_o0, kk > 0);
-            mma_commit(bar_o);
-        }
-
-        // ============================================================ T = (I + A)^{-1} Diag(beta)
-        // L = I + A, inverted in two levels of 2x2 blocks.  16x16 diagonal inverses L_II^{-1}
-        // by right-looking forward substitution (one column per thread); then each 32x32 half
-        //     [[L_a, 0], [A_ba, L_b]]^{-1} = [[L_a^{-1}, 0], [-L_b^{-1} A_ba L_a^{-1}, L_b^{-1}]]
-        // and the same rule once more for the 64x64 matrix with 32x32 blocks.  Every product
-        // is a full-precision fp32 dot product (16x16 blocks: one output per thread; 32x32
-        // blocks: 4 rows x 1 column per thread).  Scratch (P, Q) lives in A's unused
-        // upper-right 32x32 block.
-        if (tid < 64) {
-            const int Ib = tid >> 4, col = tid & 15;
-            float x[16];
+        // ============================================================ T (warps 0..7) || Y = K^ S (warps 8..15)
+        // Warps 0..7 invert L = I + A and form T (named barrier 1).  Warps 8..15 (named barrier
+        // 2) issue the O init, split the chunk-start state S^T into bf16 hi + lo in tensor
+        // memory, issue Y^T = S^T K^^T (one bf16 MMA chain per part, fp32 accumulate) and split
+        // Y^T the same way.  After both:  U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T, i.e.
+        // U = T (V - K^ S) = U~ - W S, with S entering at about 2^-16 relative precision.
+        if (warp < 8) {
+            // L = I + A, inverted in two levels of 2x2 blocks.  16x16 diagonal inverses
+            // L_II^{-1} by right-looking forward substitution (one column per thread); then each
+            // 32x32 half  [[L_a, 0], [A_ba, L_b]]^{-1} = [[L_a^{-1}, 0], [-L_b^{-1} A_ba L_a^{-1}, L_b^{-1}]]
+            // and the same rule once more for the 64x64 matrix with 32x32 blocks.  Every product
+            // is a full-precision fp32 dot product (16x16 blocks: one output per thread and
+            // half; 32x32 blocks: 4 rows x 1 column per thread).  Scratch (P, Q) lives in A's
+            // unused upper-right 32x32 block.
+            if (tid < 64) {
+                const int Ib = tid >> 4, col = tid & 15;
+                float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.0f : 0.0f;
+                for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.0f : 0.0f;
 #pragma unroll
-            for (int m = 0; m < 15; ++m)
+                for (int m = 0; m < 15; ++m)
 #pragma unroll
-                for (int r = m + 1; r < 16; ++r) x[r] -= A32[aidx(16 * Ib + r, 16 * Ib + m)] * x[m];
+                    for (int r = m + 1; r < 16; ++r) x[r] -= A32[aidx(16 * Ib + r, 16 * Ib + m)] * x[m];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) LINV[aidx(16 * Ib + r, 16 * Ib + col)] = x[r];
-        }
-        __syncthreads();
-        // dot16(X, xr, xc, Y, yr, yc): sum_m X[xr][xc + m] Y[yr + m][yc], m < 16
-        auto dot16 = [&](const float *Xm, int xr, int xc, const float *Ym, int yr, int yc) -> float {
-            float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 xv = *(const float4 *)(Xm + aidx(xr, xc + m4));
-                s0 += xv.x * Ym[aidx(yr + m4 + 0, yc)] + xv.z * Ym[aidx(yr + m4 + 2, yc)];
-                s1 += xv.y * Ym[aidx(yr + m4 + 1, yc)] + xv.w * Ym[aidx(yr + m4 + 3, yc)];
+                for (int r = 0; r < 16; ++r) LINV[aidx(16 * Ib + r, 16 * Ib + col)] = x[r];
             }
-            return s0 + s1;
-        };
-        {
-            // 32x32 halves h = 0 (blocks 0, 1) and h = 1 (blocks 2, 3):
-            // P_h = A_{2h+1,2h} L_{2h}^{-1}  ->  scratch rows 0..15, columns 32 + 16 h ..
-            const int hh = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
-            const int ra = 32 * hh, rb = 32 * hh + 16;
-            A32[aidx(r, 32 + 16 * hh + c)] = dot16(A32, rb + r, ra, LINV, ra, ra + c);
-            __syncthreads();
-            // T_{2h+1,2h} = -L_{2h+1}^{-1} P_h; the (2h, 2h+1) block is zero
-            LINV[aidx(rb + r, ra + c)] = -dot16(LINV, rb + r, rb, A32, 0, 32 + 16 * hh + c);
-            LINV[aidx(ra + r, rb + c)] = 0.0f;
-            __syncthreads();
-        }
-        {
-            // Q = A_{[2,3],[0,1]} L_{[0,1]}^{-1}: 4 rows x 1 column per thread (256 threads)
-            const int c = tid & 31, rg = (tid >> 5) & 7;   // rows 4 rg .. 4 rg + 3 of 32
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (tid < 256) {
+            named_bar_sync(1, 256);
+            // dot16(X, xr, xc, Y, yr, yc): sum_m X[xr][xc + m] Y[yr + m][yc], m < 16
+            auto dot16 = [&](const float *Xm, int xr, int xc, const float *Ym, int yr, int yc) -> float {
+                float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float4 xv = *(const float4 *)(Xm + aidx(xr, xc + m4));
+                    s0 += xv.x * Ym[aidx(yr + m4 + 0, yc)] + xv.z * Ym[aidx(yr + m4 + 2, yc)];
+                    s1 += xv.y * Ym[aidx(yr + m4 + 1, yc)] + xv.w * Ym[aidx(yr + m4 + 3, yc)];
+                }
+                return s0 + s1;
+            };
+            {
+                // halves h = 0 (blocks 0, 1) and h = 1 (blocks 2, 3):
+                // P_h = A_{2h+1,2h} L_{2h}^{-1}  ->  scratch rows 0..15, columns 32 + 16 h ..
+                const int r = tid >> 4, c = tid & 15;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    A32[aidx(r, 32 + 16 * hh + c)] = dot16(A32, 32 * hh + 16 + r, 32 * hh, LINV, 32 * hh, 32 * hh + c);
+                named_bar_sync(1, 256);
+                // T_{2h+1,2h} = -L_{2h+1}^{-1} P_h; the (2h, 2h+1) block is zero
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int ra = 32 * hh, rb = ra + 16;
+                    LINV[aidx(rb + r, ra + c)] = -dot16(LINV, rb + r, rb, A32, 0, 32 + 16 * hh + c);
+                    LINV[aidx(ra + r, rb + c)] = 0.0f;
+                }
+                named_bar_sync(1, 256);
+            }
+            {
+                // Q = A_{[2,3],[0,1]} L_{[0,1]}^{-1}: 4 rows x 1 column per thread
+                const int c = tid & 31, rg = tid >> 5;   // rows 4 rg .. 4 rg + 3 of 32
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int m4 = 0; m4 < 32; m4 += 4) {
                     float y[4];
@@ -651,10 +651,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) A32[aidx(4 * rg + q, 32 + c)] = acc[q];
-            }
-            __syncthreads();
-            // T_{[2,3],[0,1]} = -L_{[2,3]}^{-1} Q
-            if (tid < 256) {
+                named_bar_sync(1, 256);
+                // T_{[2,3],[0,1]} = -L_{[2,3]}^{-1} Q
 #pragma unroll
                 for (int q = 0; q < 4; ++q) acc[q] = 0.0f;
 #pragma unroll
@@ -670,65 +668,104 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) LINV[aidx(32 + 4 * rg + q, c)] = -acc[q];
+                named_bar_sync(1, 256);
             }
-            __syncthreads();
-        }
-        {
-            // T = L^{-1} Diag(beta), lower triangle, bf16 K-major [i][j]
-            const int i = tid >> 3, jc = tid & 7;
-            const float4 l0 = *(const float4 *)(LINV + aidx(i, 8 * jc)), l1 = *(const float4 *)(LINV + aidx(i, 8 * jc + 4));
-            const float4 b0 = *(const float4 *)(BETAsm + 8 * jc), b1 = *(const float4 *)(BETAsm + 8 * jc + 4);
-            const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float vals[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) vals[e] = 8 * jc + e <= i ? lv[e] * bv[e] : 0.0f;
-            *(uint4 *)(sm + OFF_T + swz(i, jc)) = pack8(vals);
+            for (int it = 0; it < 2; ++it) {
+                // T = L^{-1} Diag(beta), lower triangle, bf16 K-major [i][j]
+                const int idx = tid + 256 * it, i = idx >> 3, jc = idx & 7;
+                const float4 l0 = *(const float4 *)(LINV + aidx(i, 8 * jc)), l1 = *(const float4 *)(LINV + aidx(i, 8 * jc + 4));
+                const float4 b0 = *(const float4 *)(BETAsm + 8 * jc), b1 = *(const float4 *)(BETAsm + 8 * jc + 4);
+                const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                float vals[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vals[e] = 8 * jc + e <= i ? lv[e] * bv[e] : 0.0f;
+                *(uint4 *)(sm + OFF_T + swz(i, jc)) = pack8(vals);
+            }
+            fence_proxy_async();
+        } else {
+            const int hb = (warp - 8) >> 2;   // column half of the TMEM tiles this warp splits
+            if (tid == NT - 32) {
+                // O^T = S^T Q^^T at tf32 (A = fp32 state in TMEM, 8 key channels per MMA); it
+                // completes on bar_o before the state is decayed
+                tc_fence_after();
+                const uint32_t sQ = smem_u32(sm + OFF_QH);
+                for (int kk = 0; kk < 16; ++kk)
+                    mma_ts_tf32(tmem + TM_O, tmem + TM_S + kk * 8, sdesc(sQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                id_o0, kk > 0);
+                mma_commit(bar_o);
+            }
+            // S^T (fp32, key channels 64 hb .. 64 hb + 63) -> bf16 hi + lo, two per column
+#pragma unroll
+            for (int cc = 0; cc < 64; cc += 32) {
+                uint32_t r[32], hi[16], lo[16];
+                tmem_ld32(tmem + lane_q + TM_S + 64 * hb + cc, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                    hi[e] = pack_bf16x2(x0, x1);
+                    const float2 hv = unpack_bf16x2(hi[e]);
+                    lo[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
+                }
+                tmem_st16(tmem + lane_q + TM_SH + 32 * hb + cc / 2, hi);
+                tmem_st16(tmem + lane_q + TM_SL + 32 * hb + cc / 2, lo);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar_sync(2, 256);
+            if (tid == 256) {
+                // Y^T = S_hi^T K^^T + S_lo^T K^^T  (K^ = Gamma k, bf16 K-major in the stage)
+                tc_fence_after();
+                const uint32_t sK = smem_u32(stg + ST_K);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + TM_Y, tmem + TM_SH + kk * 8, sdesc(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                           id_op, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + TM_Y, tmem + TM_SL + kk * 8, sdesc(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                           id_op, 1);
+                mma_commit(bar_y);
+            }
+            if (mbar_wait_bounded(bar_y, (uint32_t)(n & 1), abort_flag, p.err)) {
+                tc_fence_after();
+                // Y^T (fp32, tokens 32 hb .. 32 hb + 31) -> bf16 hi + lo
+                uint32_t r[32], hi[16], lo[16];
+                tmem_ld32(tmem + lane_q + TM_Y + 32 * hb, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                    hi[e] = pack_bf16x2(x0, x1);
+                    const float2 hv = unpack_bf16x2(hi[e]);
+                    lo[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
+                }
+                tmem_st16(tmem + lane_q + TM_HI32 + 16 * hb, hi);
+                tmem_st16(tmem + lane_q + TM_LO32 + 16 * hb, lo);
+                tmem_wait_st();
+            }
         }
-        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (*abort_flag) break;
 
-        // ============================================================ W^T = K^^T T^T, U~^T = V^T T^T
+        // ============================================================ U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t sK = smem_u32(stg + ST_K), sV = smem_u32(stg + ST_V), sT_ = smem_u32(sm + OFF_T);
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + TM_W, sdesc(sK + kk * 2048, 8192, 1024), sdesc(sT_ + kk * 32, 16, 1024), id_wt, kk > 0);
+            const uint32_t sV = smem_u32(stg + ST_V), sT_ = smem_u32(sm + OFF_T);
             for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tmem + TM_U, sdesc(sV + kk * 2048, 8192, 1024), sdesc(sT_ + kk * 32, 16, 1024), id_wt, kk > 0);
-            mma_commit(bar_mma);
-        }
-        if (!mma_wait()) break;
-        tc_fence_after();
-        {
-            // W^T (lane = key channel c = 32 lq + lane) -> W in shared memory, fp32 K-major [i][c];
-            // K-block c / 32 = this warp's lane quarter; one 128-byte row per token i
-            uint32_t r[16];
-            tmem_ld16(tmem + lane_q + TM_W + 16 * cg, r);
-            tmem_wait_ld();
-            uint8_t *wb = sm + OFF_W + lq * 8192 + (lane & 3) * 4;
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                *(uint32_t *)(wb + swz(16 * cg + e, lane >> 2)) = r[e];
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            // U^T -= S^T W^T at tf32: A = fp32 state in TMEM, B = W fp32 K-major
-            const uint32_t sW = smem_u32(sm + OFF_W);
-            for (int kk = 0; kk < 16; ++kk)
-                mma_ts_tf32(tmem + TM_U, tmem + TM_S + kk * 8, sdesc(sW + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                            id_u, 1);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts(tmem + TM_U, tmem + TM_HI32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, 1);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts(tmem + TM_U, tmem + TM_LO32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, 1);
             mma_commit(bar_mma);
         }
         if (!mma_wait()) break;
         if (!mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err)) break;
         tc_fence_after();
         {
-            // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column)
+            // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column; Y's are consumed)
             uint32_t r[16], r8[8], l8[8];
             tmem_ld16(tmem + lane_q + TM_U + 16 * cg, r);
             tmem_wait_ld();
@@ -739,10 +776,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float2 hv = unpack_bf16x2(r8[e]);
                 l8[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
             }
-            tmem_st8(tmem + lane_q + TM_UB + 8 * cg, r8);
-            tmem_st8(tmem + lane_q + TM_UL + 8 * cg, l8);
-            // S^T <- S^T Diag(exp G_C) (every reader of the chunk-start state has finished: the
-            // O init was waited for above)
+            tmem_st8(tmem + lane_q + TM_HI32 + 8 * cg, r8);
+            tmem_st8(tmem + lane_q + TM_LO32 + 8 * cg, l8);
+            // S^T <- S^T Diag(exp G_C) (every reader of the chunk-start state has finished)
             uint32_t sr[32];
             const uint32_t ta = tmem + lane_q + TM_S + 32 * cg;
             tmem_ld32(ta, sr);
@@ -758,13 +794,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             const uint32_t sP = smem_u32(stg + ST_P), sPL = smem_u32(stg + ST_PL), sG = smem_u32(stg + ST_G);
             for (int kk = 0; kk < 4; ++kk) {
-                mma_ts(tmem + TM_O, tmem + TM_UB + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
-                mma_ts(tmem + TM_O, tmem + TM_UL + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
-                mma_ts(tmem + TM_O, tmem + TM_UB + kk * 8, sdesc(sPL + kk * 32, 16, 1024), id_op, 1);
+                mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
+                mma_ts(tmem + TM_O, tmem + TM_LO32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
+                mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sPL + kk * 32, 16, 1024), id_op, 1);
             }
             for (int kk = 0; kk < 4; ++kk) {
-                mma_ts(tmem + TM_S, tmem + TM_UB + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
-                mma_ts(tmem + TM_S, tmem + TM_UL + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
+                mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
+                mma_ts(tmem + TM_S, tmem + TM_LO32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
             }
             mma_commit(bar_mma);
         }
