@@ -582,8 +582,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ============================================================ T (warps 0..7) || Y = K^ S (warps 8..15)
         // Warps 0..7 invert L = I + A and form T (named barrier 1).  Warps 8..15 (named barrier
         // 2) issue the O init, split the chunk-start state S^T into bf16 hi + lo in tensor
-        // memory, issue Y^T = S^T K^^T (one bf16 MMA chain per part, fp32 accumulate) and split
-        // Y^T the same way.  After both:  U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T, i.e.
+        // memory, issue Y^T = S^T K^^T (one bf16 MMA chain per part, fp32 accumulate), split
+        // Y^T the same way and decay the state by exp(G_C).  After both:  U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T, i.e.
         // U = T (V - K^ S) = U~ - W S, with S entering at about 2^-16 relative precision.
         if (warp < 8) {
             // L = I + A, inverted in two levels of 2x2 blocks.  16x16 diagonal inverses
@@ -744,6 +744,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_st16(tmem + lane_q + TM_LO32 + 16 * hb, lo);
                 tmem_wait_st();
             }
+            // S^T <- S^T Diag(exp G_C): every reader of the chunk-start state is done once the
+            // O init has completed (the split above and the Y MMAs read the copies)
+            if (mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err)) {
+                tc_fence_after();
+#pragma unroll
+                for (int cc = 0; cc < 64; cc += 32) {
+                    uint32_t sr[32];
+                    const uint32_t ta = tmem + lane_q + TM_S + 64 * hb + cc;
+                    tmem_ld32(ta, sr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sr[e] = __float_as_uint(__uint_as_float(sr[e]) * GCsm[64 * hb + cc + e]);
+                    tmem_st32(ta, sr);
+                }
+                tmem_wait_st();
+            }
         }
         tc_fence_before();
         __syncthreads();
@@ -762,7 +778,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mma_commit(bar_mma);
         }
         if (!mma_wait()) break;
-        if (!mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err)) break;
         tc_fence_after();
         {
             // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column; Y's are consumed)
@@ -778,14 +793,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tmem_st8(tmem + lane_q + TM_HI32 + 8 * cg, r8);
             tmem_st8(tmem + lane_q + TM_LO32 + 8 * cg, l8);
-            // S^T <- S^T Diag(exp G_C) (every reader of the chunk-start state has finished)
-            uint32_t sr[32];
-            const uint32_t ta = tmem + lane_q + TM_S + 32 * cg;
-            tmem_ld32(ta, sr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sr[e] = __float_as_uint(__uint_as_float(sr[e]) * GCsm[32 * cg + e]);
-            tmem_st32(ta, sr);
             tmem_wait_st();
         }
         tc_fence_before();
