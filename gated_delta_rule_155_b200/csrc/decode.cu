@@ -9,8 +9,8 @@
 // The state is read once and written once.  Value columns are independent, so a CTA
 // owns one 64-column slice of one head: 256 threads, 16 threads per row segment of
 // 64 floats (one float4 each, fully coalesced 256-byte row segments), 16 rows per
-// pass, dk/16 passes.  Each thread keeps its dk/16 decayed float4s in registers
-// between the reduction and the write-back.  Column sums over dk reduce first
+// pass, dk/16 passes, issued before anything else.  Each thread keeps its dk/16 decayed
+// float4s in registers between the reduction and the write-back; three CTAs fit per SM.  Column sums over dk reduce first
 // across the two rows a warp holds (shuffle) and then across the 8 warps (smem).
 #include "common.cuh"
 #include "internal.h"
@@ -22,7 +22,7 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_SLICE = 64;  // value columns per CTA
 
 template <typename IO, int DK>
-__global__ void __launch_bounds__(DEC_THREADS)
+__global__ void __launch_bounds__(DEC_THREADS, 3)
 kda_decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                   const IO *__restrict__ g, const IO *__restrict__ beta, float *state,
                   IO *__restrict__ out, int H, int dv)
@@ -42,6 +42,17 @@ kda_decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *
     const size_t kvec = (size_t)bh * DK;
     const size_t vvec = (size_t)bh * dv;
 
+    // the state loads go out first, so their latency overlaps the small vector loads below
+    const int col = (tid & 15) * 4;       // column offset inside the slice
+    const int row0 = tid >> 4;            // 0..15
+    float *Sbase = state + (size_t)bh * DK * dv + v0 + col;
+    float4 s[NPASS];
+#pragma unroll
+    for (int p = 0; p < NPASS; ++p) {
+        const int r = row0 + p * ROWS_PER_PASS;
+        s[p] = *reinterpret_cast<const float4 *>(Sbase + (size_t)r * dv);
+    }
+
     if (tid < DK) {
         s_alpha[tid] = __expf(to_f32(g[kvec + tid]));
         s_k[tid] = to_f32(k[kvec + tid]);
@@ -55,17 +66,7 @@ kda_decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *
         if (lane == 0) s_qk = p;
     }
 
-    const int col = (tid & 15) * 4;       // column offset inside the slice
-    const int row0 = tid >> 4;            // 0..15
-    float *Sbase = state + (size_t)bh * DK * dv + v0 + col;
-
-    float4 s[NPASS];
     float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int p = 0; p < NPASS; ++p) {
-        const int r = row0 + p * ROWS_PER_PASS;
-        s[p] = *reinterpret_cast<const float4 *>(Sbase + (size_t)r * dv);
-    }
 #pragma unroll
     for (int p = 0; p < NPASS; ++p) {
         const int r = row0 + p * ROWS_PER_PASS;
