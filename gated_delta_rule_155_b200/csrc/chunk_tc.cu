@@ -78,11 +78,11 @@ constexpr int AST = 68;
 constexpr int OFF_A32 = OFF_X2;
 constexpr int OFF_LINV = OFF_X2 + 64 * AST * 4;
 // per-(block, channel) table, fp32 rows of FSTRIDE (128 channels + padding that puts the
-// four blocks of one channel in different banks): fG, fL, fM, block log-decay L_B and
-// first-half log-decay H_B (tokens 0..7 of the block) for blocks 0..3, then fC for the six
-// (B, I) pairs with I > B
+// four blocks of one channel in different banks): fG, fL, fM for blocks 0..3, the half-block
+// log-decays (row FT_HS + 2 B + half: sum of g over tokens 8 half .. 8 half + 7 of block B),
+// then fC for the six (B, I) pairs with I > B
 constexpr int FSTRIDE = 136;
-constexpr int FT_G = 0, FT_L = 4, FT_M = 8, FT_LB = 12, FT_H8 = 16, FT_C = 20;   // row numbers
+constexpr int FT_G = 0, FT_L = 4, FT_M = 8, FT_HS = 12, FT_C = 20;   // row numbers
 constexpr int FT_BYTES = 26 * FSTRIDE * 4;
 constexpr int OFF_FT = OFF_X2 + 32768;
 constexpr int OFF_T = OFF_FT + 2048;             // past L^{-1}'s overhang, 1024-aligned
@@ -269,44 +269,71 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         constexpr float INV_SC = 7.523164e-37f;    // SC = 2^120, INV_SC = 2^-120
         constexpr float LN_SC = 83.17766f;         // 120 ln 2
-        // pass 1, one (block, channel) per thread: block log-decay L_B (sum of g over the 16
-        // tokens), its first-half part H_B, and the factors
+        // Token mapping of passes A and C: warp (pr, cq, th) takes token position pp = lane & 7
+        // of the half th of block pr (s = 0) and of block 3 - pr (s = 1), so every warp carries
+        // the same number of later-block Gram columns; lane >> 3 picks 8 of the 32 channels of
+        // quarter cq.
+        const int pr = warp & 1;
+        const int cq = (warp >> 1) & 3;   // channel quarter (32 channels)
+        const int th = warp >> 3;         // token half of the block
+        const int pp = lane & 7;          // token position inside the half
+        const int a = 4 * (cq & 1) + (lane >> 3);   // 16-byte chunk inside the channel block
+        const int cb = cq >> 1;           // channel block (64 channels)
+        const int c0 = 64 * cb + 8 * a;
+        auto ftab = [&](int row, float (&f)[8]) {
+            const float *src = FT + row * FSTRIDE + c0;
+            const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
+            f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+        };
+        // pass A: in-half inclusive prefix of g by an 8-lane scan; the last lane of each half
+        // publishes the half-block sums
+        float Gh[2][8];
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            const int B = s == 0 ? pr : 3 - pr;
+            const int i = 16 * B + 8 * th + pp;
+            unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), Gh[s]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float l = Gh[s][e];
+                float y = __shfl_up_sync(0xffffffffu, l, 1, 8);
+                if (pp >= 1) l += y;
+                y = __shfl_up_sync(0xffffffffu, l, 2, 8);
+                if (pp >= 2) l += y;
+                y = __shfl_up_sync(0xffffffffu, l, 4, 8);
+                if (pp >= 4) l += y;
+                Gh[s][e] = l;
+            }
+            if (pp == 7) {
+                float *dst = FT + (FT_HS + 2 * B + th) * FSTRIDE + c0;
+                *(float4 *)dst = make_float4(Gh[s][0], Gh[s][1], Gh[s][2], Gh[s][3]);
+                *(float4 *)(dst + 4) = make_float4(Gh[s][4], Gh[s][5], Gh[s][6], Gh[s][7]);
+            }
+        }
+        __syncthreads();
+        // pass B, one (block, channel) per thread: block log-decays L_J and the factors
         //   fG = exp(G_blockstart)      fL = exp(G_C - G_blockend)
         //   fM = exp(-L_B / 2) / SC     (block-start reference, 1 / SC, where L_B < BAD_LOG)
         //   fC(B, I) = exp(m_I - G_blockend of B) for later blocks I > B, m_I the reference of I.
         // All exponents are sums of non-positive log-decays (plus L_B / 2 >= -84 for fM), so a
         // factor underflows only where the exact value does.
         {
-            const int c = tid >> 2, Bq = tid & 3;
-            const uint8_t *gcol = stg + ST_G + (c >> 6) * 8192 + ((c & 7) << 1);
-            const int chk = (c & 63) >> 3;
-            float h0 = 0.0f, h1 = 0.0f;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                // token order rotated by the block, so the four blocks' rows read by one warp
-                // instruction fall in different banks
-                const int tt = (t + 2 * Bq) & 15;
-                const float x = __bfloat162float(*(const __nv_bfloat16 *)(gcol + swz(16 * Bq + tt, chk)));
-                if (tt < 8) h0 += x;
-                else h1 += x;
-            }
-            const float L = h0 + h1;
+            const int c = tid & 127, Bq = tid >> 7;
             float Lv[4];
 #pragma unroll
-            for (int J = 0; J < 4; ++J) Lv[J] = __shfl_sync(0xffffffffu, L, (lane & ~3) | J);
-            float lpre = 0.0f, lpost = 0.0f;
+            for (int J = 0; J < 4; ++J) Lv[J] = FT[(FT_HS + 2 * J) * FSTRIDE + c] + FT[(FT_HS + 2 * J + 1) * FSTRIDE + c];
+            float lpre = 0.0f, lpost = 0.0f, L = 0.0f;
 #pragma unroll
             for (int J = 0; J < 4; ++J) {
                 if (J < Bq) lpre += Lv[J];
                 if (J > Bq) lpost += Lv[J];
+                if (J == Bq) L = Lv[J];
             }
             const bool badB = !(L >= BAD_LOG);
             float *ft = FT + Bq * FSTRIDE + c;
             ft[FT_G * FSTRIDE] = __expf(lpre);
             ft[FT_L * FSTRIDE] = __expf(lpost);
             ft[FT_M * FSTRIDE] = __expf((badB ? 0.0f : -0.5f * L) - LN_SC);
-            ft[FT_LB * FSTRIDE] = L;
-            ft[FT_H8 * FSTRIDE] = h0;
             if (badB) atomicOr(&badmask[Bq * 4 + (c >> 5)], 1u << (c & 31));
 #pragma unroll
             for (int I = 1; I < 4; ++I) {
@@ -320,27 +347,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (Bq == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
         }
         __syncthreads();
-        // pass 2, per token.  Warp (pr, cq, th) takes token position p = lane & 7 of the half th
-        // of block pr (s = 0) and of block 3 - pr (s = 1), so every warp carries the same
-        // number of later-block Gram columns; lane >> 3 picks 8 of the 32 channels of quarter
-        // cq.  With SC = 2^120:
+        // pass C, per token.  With SC = 2^120:
         //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
         //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
         // from log-domain prefix sums, so no partial product can underflow; both are normal
         // numbers for block log-decays down to BAD_LOG (SC e^-168 ~ e^-84.8).
         {
-            const int pr = warp & 1;
-            const int cq = (warp >> 1) & 3;   // channel quarter (32 channels)
-            const int th = warp >> 3;         // token half of the block
-            const int pp = lane & 7;          // token position inside the half
-            const int a = 4 * (cq & 1) + (lane >> 3);   // 16-byte chunk inside the channel block
-            const int cb = cq >> 1;           // channel block (64 channels)
-            const int c0 = 64 * cb + 8 * a;
-            auto ftab = [&](int row, float (&f)[8]) {
-                const float *src = FT + row * FSTRIDE + c0;
-                const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
-                f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
-            };
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
                 const int B = s == 0 ? pr : 3 - pr;
@@ -348,23 +360,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t off = cb * 8192 + swz(i, a);
                 float Gin[8], Lb[8];
                 {
-                    // G_i - G_blockstart: inclusive scan over the 8 lanes of the half, plus H_B
-                    // for the second half
-                    float hb[8];
-                    ftab(FT_H8 + B, hb);
-                    unpack8(*(const uint4 *)(stg + ST_G + off), Gin);
+                    // G_i - G_blockstart = in-half prefix (+ the first half's sum); L_B
+                    float h0[8], h1[8];
+                    ftab(FT_HS + 2 * B, h0);
+                    ftab(FT_HS + 2 * B + 1, h1);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        float l = Gin[e];
-                        float y = __shfl_up_sync(0xffffffffu, l, 1, 8);
-                        if (pp >= 1) l += y;
-                        y = __shfl_up_sync(0xffffffffu, l, 2, 8);
-                        if (pp >= 2) l += y;
-                        y = __shfl_up_sync(0xffffffffu, l, 4, 8);
-                        if (pp >= 4) l += y;
-                        Gin[e] = l + (th ? hb[e] : 0.0f);
+                        Gin[e] = Gh[s][e] + (th ? h0[e] : 0.0f);
+                        Lb[e] = h0[e] + h1[e];
                     }
-                    ftab(FT_LB + B, Lb);
                 }
                 const uint32_t badbits = (badmask[B * 4 + (c0 >> 5)] >> (c0 & 31)) & 0xffu;
                 float qf[8], kf[8], o[8], E1[8], E2[8], f[8];
