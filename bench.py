@@ -358,7 +358,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and ws == 1 and "cpu" not in skip:
-        cpu = cpu_baseline_prefill(steps=1)
+        cpu = cpu_baseline_prefill()
 
     gpu_launches = args.steps * launches_per["prefill"] + launches_per.get("decode", 0) + \
         launches_per.get("layer", 0)
@@ -384,10 +384,11 @@ def run_ours(args):
 # ----------------------------------------------------------------------------- oracle (CPU)
 
 
-def cpu_baseline_prefill(steps=1):
+def cpu_baseline_prefill(min_seconds=10.0, max_reps=40):
     """The fp64 oracle, as it stands, on a bounded sample of the prefill workload: n heads of
-    the T = 8192 sequences (heads are independent), all host threads.  Returns the
-    cpu_baseline object; value in tokens/s of the full 96-head workload."""
+    the T = 8192 sequences (heads are independent), all host threads, run repeatedly until
+    about `min_seconds` of CPU work have been timed.  Returns the cpu_baseline object; value
+    in tokens/s of the full 96-head workload."""
     import oracle
     from gated_delta_rule_155_b200 import inputs
 
@@ -396,16 +397,17 @@ def cpu_baseline_prefill(steps=1):
     nh = int(min(96, max(8, 2 * cores)))
     d = inputs.prefill_inputs(1, w["T"], nh, w["dk"], w["dv"], io=w["io"], seed=w["seed"])
     arrs = [d[n].double().numpy() for n in ("q", "k", "v", "g", "beta")]
-    best = math.inf
-    for _ in range(steps):
+    reps, total = 0, 0.0
+    while reps < max_reps and (total < min_seconds or reps == 0):
         t0 = time.perf_counter()
         oracle.recurrent(*arrs, None, nthreads=cores)
-        best = min(best, time.perf_counter() - t0)
-    token_heads = nh * w["T"]
-    return {"value": round(token_heads / best / w["H"], 2), "unit": "tokens/s", "cores": cores,
+        total += time.perf_counter() - t0
+        reps += 1
+    token_heads = nh * w["T"] * reps
+    return {"value": round(token_heads / total / w["H"], 2), "unit": "tokens/s", "cores": cores,
             "kind": "oracle",
-            "sample": f"{nh} heads x T={w['T']} of the prefill workload (fp64 token recurrence, "
-                      f"{token_heads} token-heads, {best:.2f} s); tokens/s = token-heads/s / 96"}
+            "sample": f"{reps} runs of {nh} heads x T={w['T']} of the prefill workload (fp64 token "
+                      f"recurrence, {token_heads} token-heads, {total:.1f} s); tokens/s = token-heads/s / 96"}
 
 
 def run_reference(args):
