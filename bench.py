@@ -6,8 +6,9 @@
 Headline (`value`): chunked-prefill throughput, tokens/s over all N GPUs, on the
 H = 96, d = 128 prefill workload (B=4, T=8192, chunk 64, bf16 I/O, fp32 state).
 A step is one kda_forward_chunked call over that batch.  The same line carries the
-decode workload (B=256, H=96, 20 chained in-place steps; GB/s of state traffic) and
-the full layer workload (B=2, T=16384; tokens/s), each with its roofline.
+decode workload (B=256, H=96, 20 chained in-place steps; GB/s of state traffic), the
+layer decode step with its conv cache on the same shape, and the full layer workload
+(B=2, T=16384; tokens/s), each with its roofline.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of the
 workload (heads and sequences are independent — no data-path collective), a barrier
@@ -58,7 +59,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--skip", default="", help="comma list of: decode,layer,e2e,cpu")
+    ap.add_argument("--skip", default="", help="comma list of: decode,layer_decode,layer,e2e,cpu")
     return ap.parse_args()
 
 
@@ -318,6 +319,48 @@ def run_ours(args):
         del state, steps_in, od, dd
         torch.cuda.empty_cache()
 
+    # ------------------------------------------------------------------ layer decode (conv cache)
+    if "layer_decode" not in skip:
+        wd = inputs.WORKLOADS[DECODE]
+        Bd, Hd, dd_ = wd["B"], wd["H"], wd["dk"]
+        Ld = inputs.layer_inputs(Bd, wd["steps"], Hd, dd_, dd_, io=wd["io"], seed=wd["seed"], conv_std=0.5,
+                                 s0_std=wd["s0_std"])
+        to = lambda x: None if x is None else x.contiguous().to(dev)
+        state = to(Ld["s0"])
+        caches = [torch.zeros((Bd, 3, Hd * dd_), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        fixed = {n: to(Ld[n]) for n in ("conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "o_norm_w")}
+        steps_in = [{n: to(Ld[n][:, t]) for n in ("q_raw", "k_raw", "v_raw", "g_raw", "b_raw", "o_gate_raw")}
+                    for t in range(wd["steps"])]
+        od = torch.empty((Bd, Hd, dd_), dtype=torch.bfloat16, device=dev)
+
+        def layer_decode_run():
+            for x in steps_in:
+                kda.kda_layer_decode_step(x["q_raw"], x["k_raw"], x["v_raw"], fixed["conv_q"], fixed["conv_k"],
+                                          fixed["conv_v"], *caches, x["g_raw"], fixed["A_log"], fixed["dt_bias"],
+                                          x["b_raw"], x["o_gate_raw"], state, fixed["o_norm_w"], out=od,
+                                          stream=stream)
+
+        reps = max(1, args.steps // 10)
+        total_ld, _ = timed(torch, layer_decode_run, reps, max(1, args.warmup // 3), stream, barrier,
+                            per_launch=False)
+        kda.kda_check_device_error(stream)
+        ms_ld = max_over_ranks(total_ld / (reps * wd["steps"]))
+        state_bytes = 2 * Bd * Hd * dd_ * dd_ * 4
+        # raw q, k, v, g, gate and out (bf16), beta, the three caches read and written
+        io_bytes = Bd * Hd * (6 * dd_ * 2 + 2 + 2 * 3 * 3 * dd_ * 2)
+        gbs = (state_bytes + io_bytes) / (ms_ld / 1e3) / 1e9
+        res["layer_decode"] = {
+            "workload": "kda_layer_decode_step B=256 H=96 dk=dv=128 bf16 (conv cache + prologue + recurrence + "
+                        "epilogue), fp32 state in place, 20 chained steps",
+            "value": round(ws * gbs, 1), "unit": "GB/s", "ms_per_step": round(ms_ld, 4),
+            "tokens_per_s": round(ws * Bd / (ms_ld / 1e3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                         "kernel": "kda_layer_decode", "bytes_per_launch": state_bytes + io_bytes}}
+        launches_per["layer_decode"] = wd["steps"] * reps
+        del state, caches, steps_in, od, Ld, fixed
+        torch.cuda.empty_cache()
+
     # ------------------------------------------------------------------ layer
     if "layer" not in skip:
         wl = inputs.WORKLOADS[LAYER]
@@ -361,7 +404,7 @@ def run_ours(args):
         cpu = cpu_baseline_prefill()
 
     gpu_launches = args.steps * launches_per["prefill"] + launches_per.get("decode", 0) + \
-        launches_per.get("layer", 0)
+        launches_per.get("layer_decode", 0) + launches_per.get("layer", 0)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

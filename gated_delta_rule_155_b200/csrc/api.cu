@@ -181,6 +181,31 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
     return cuda_status(kda::launch_epilogue(ea, s));
 }
 
+kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const void *v_raw,
+                                   const float *conv_q, const float *conv_k, const float *conv_v,
+                                   void *cache_q, void *cache_k, void *cache_v, const void *g_raw,
+                                   const float *A_log, const float *dt_bias, const void *b_raw,
+                                   const void *o_gate_raw, const float *o_norm_w, float norm_eps,
+                                   float *state, void *out, int B, int H, int dk, int dv,
+                                   kda_dtype_t io, kda_stream_t stream)
+{
+    kda_status_t st = check_dims(B, 1, H, dk, dv, io);
+    if (st != KDA_OK) return st;
+    if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (!(norm_eps >= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !cache_q || !cache_k || !cache_v ||
+        !g_raw || !A_log || !b_raw || !o_gate_raw || !state || !out)
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cache_q, cache_k, cache_v, g_raw,
+                          A_log, dt_bias, b_raw, o_gate_raw, o_norm_w, state, out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    kda::LayerDecodeArgs a{q_raw, k_raw, v_raw, cache_q, cache_k, cache_v, conv_q, conv_k, conv_v,
+                           g_raw, A_log, dt_bias, b_raw, o_gate_raw, o_norm_w, norm_eps, state, out,
+                           B, H, io_of(io)};
+    return cuda_status(kda::launch_layer_decode(a, (cudaStream_t)stream));
+}
+
 kda_status_t kda_check_device_error(kda_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -49,6 +49,23 @@ struct EpilogueArgs {
     IoType io;
 };
 
+// One decode step of the whole layer core (conv cache + prologue + recurrence + epilogue).
+struct LayerDecodeArgs {
+    const void *q_raw, *k_raw, *v_raw;      // [B, H*128], io
+    void *cache_q, *cache_k, *cache_v;      // [B, 3, H*128], io, in place (oldest tap first)
+    const float *conv_q, *conv_k, *conv_v;  // [H*128, 4]
+    const void *g_raw;                      // [B, H, 128], io
+    const float *A_log, *dt_bias;           // [H]; [H*128] or null
+    const void *b_raw, *o_gate_raw;         // [B, H]; [B, H, 128], io
+    const float *gain;                      // [128] or null
+    float eps;
+    float *state;                           // [B, H, 128, 128] fp32, in place
+    void *out;                              // [B, H, 128], io
+    int B, H;
+    IoType io;
+};
+cudaError_t launch_layer_decode(const LayerDecodeArgs &a, cudaStream_t s);
+
 // CUDA-core chunked kernel: any supported dtype, dk, dv in {64, 128}.
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 // Exact fp32 chunked kernel on CUDA cores for dk = dv = 128 with all-fp32 operands.

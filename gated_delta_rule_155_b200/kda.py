@@ -51,6 +51,8 @@ def _load():
     lib.kda_layer_forward_noalloc.restype = i
     lib.kda_layer_forward_noalloc.argtypes = [vp] * 12 + [f] + [vp] * 3 + [i] * 5 + [i, vp]
     lib.kda_check_device_error.restype = i
+    lib.kda_layer_decode_step.argtypes = [vp] * 15 + [f] + [vp] * 2 + [i] * 4 + [i, vp]
+    lib.kda_layer_decode_step.restype = i
     lib.kda_check_device_error.argtypes = [vp]
     return lib
 
@@ -186,6 +188,37 @@ def kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log,
         float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(workspace),
         ws_bytes, B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward")
     return out, final_state
+
+
+def kda_layer_decode_step(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cache_q, cache_k, cache_v, g_raw,
+                          A_log, dt_bias, b_raw, o_gate_raw, state, o_norm_w=None, *, norm_eps=1e-6,
+                          out=None, stream=None):
+    """One decode step of the layer core.  ``cache_*`` [B, 3, H*d] (io dtype, oldest tap first)
+    and ``state`` [B, H, dk, dv] fp32 are updated in place.  Returns out [B, H, dv]."""
+    B, H, dk = g_raw.shape
+    dv = o_gate_raw.shape[-1]
+    io = g_raw.dtype
+    f32 = torch.float32
+    for t, s_, d, n in ((q_raw, (B, H * dk), io, "q_raw"), (k_raw, (B, H * dk), io, "k_raw"),
+                        (v_raw, (B, H * dv), io, "v_raw"), (b_raw, (B, H), io, "b_raw"),
+                        (o_gate_raw, (B, H, dv), io, "o_gate_raw"),
+                        (cache_q, (B, 3, H * dk), io, "cache_q"), (cache_k, (B, 3, H * dk), io, "cache_k"),
+                        (cache_v, (B, 3, H * dv), io, "cache_v"),
+                        (conv_q, (H * dk, 4), f32, "conv_q"), (conv_k, (H * dk, 4), f32, "conv_k"),
+                        (conv_v, (H * dv, 4), f32, "conv_v"), (A_log, (H,), f32, "A_log"),
+                        (state, (B, H, dk, dv), f32, "state")):
+        _need(t, s_, d, n)
+    _need(dt_bias, (H * dk,), f32, "dt_bias", allow_none=True)
+    _need(o_norm_w, (dv,), f32, "o_norm_w", allow_none=True)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=io, device=g_raw.device)
+    _need(out, (B, H, dv), io, "out")
+    _check(_lib.kda_layer_decode_step(
+        _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
+        _ptr(cache_q), _ptr(cache_k), _ptr(cache_v), _ptr(g_raw), _ptr(A_log), _ptr(dt_bias),
+        _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w), float(norm_eps), _ptr(state), _ptr(out),
+        B, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_decode_step")
+    return out
 
 
 def kda_layer_forward_noalloc(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,

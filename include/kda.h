@@ -158,6 +158,37 @@ kda_status_t kda_layer_forward_noalloc(const void *q_raw, const void *k_raw, con
                                        kda_dtype_t io, kda_stream_t stream);
 
 /*
+ * kda_layer_decode_step — one decode step of the layer core for B sequences: the prologue,
+ * the gated delta rule and the epilogue of kda_layer_forward for the single new token t,
+ * with the conv history kept in a cache instead of recomputed.
+ *   y = SiLU(w[c,0] x[t-3] + w[c,1] x[t-2] + w[c,2] x[t-1] + w[c,3] x[t])  per channel, for q,
+ *   k and v, x[t-3..t-1] read from the cache, which then shifts in x[t]; then as
+ *   kda_layer_forward: q, k L2-normalised, g, beta, the state update
+ *   S <- (I - beta k k^T) Diag(exp g) S + beta k v^T, o = S^T q, RMSNorm x gain x sigmoid gate.
+ * (The Kimi-K3 linear-attention config's short conv of kernel 4; the pages note that KDA
+ *  decode with a cached state is not yet implemented in the MaxText port.)
+ *   q_raw, k_raw  [B, H*dk] io dtype         v_raw        [B, H*dv] io dtype
+ *   cache_q, cache_k [B, 3, H*dk] io dtype   cache_v      [B, 3, H*dv] io dtype
+ *                 updated in place; tap 0 is the oldest token (t-3); zeros = empty history
+ *   conv_q, conv_k [H*dk, 4] fp32            conv_v       [H*dv, 4] fp32
+ *   g_raw         [B, H, dk] io dtype        A_log        [H] fp32
+ *   dt_bias       [H*dk] fp32 or NULL        b_raw        [B, H] io dtype
+ *   o_gate_raw    [B, H, dv] io dtype        o_norm_w     [dv] fp32 or NULL (ones)
+ *   state         [B, H, dk, dv] fp32, updated in place
+ *   out           [B, H, dv] io dtype (written)
+ * Supported: dk = dv = 128 (KDA_ERR_UNSUPPORTED otherwise), both dtypes.  Every pointer
+ * 16-byte aligned.  n calls from an empty cache and state give the outputs of
+ * kda_layer_forward over the same n tokens.
+ */
+kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const void *v_raw,
+                                   const float *conv_q, const float *conv_k, const float *conv_v,
+                                   void *cache_q, void *cache_k, void *cache_v, const void *g_raw,
+                                   const float *A_log, const float *dt_bias, const void *b_raw,
+                                   const void *o_gate_raw, const float *o_norm_w, float norm_eps,
+                                   float *state, void *out, int B, int H, int dk, int dv,
+                                   kda_dtype_t io, kda_stream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the library's device error word
  * (set by a kernel whose bounded wait gave up) and any sticky CUDA error.
  * Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA.

@@ -93,6 +93,23 @@ def test_decode_rejects_bad_arguments(lib):
     assert ok(v=MIS) == 3
 
 
+def test_layer_decode_rejects_bad_arguments(lib):
+    names = ["qr", "kr", "vr", "cq", "ck", "cv", "xq", "xk", "xv", "g", "al", "dt", "b", "z", "w"]
+
+    def step(eps=1e-6, **kw):
+        ptrs = [kw.get(n, None if n in ("dt", "w") else A16) for n in names]
+        return lib.kda_layer_decode_step(*ptrs, ctypes.c_float(eps), kw.get("S", A16), kw.get("o", A16),
+                                         kw.get("B", 2), kw.get("H", 3), kw.get("dk", 128), kw.get("dv", 128),
+                                         kw.get("io", 1), None)
+    assert step(S=None) == 1
+    assert step(xk=None) == 1
+    assert step(eps=-1.0) == 1
+    assert step(H=0) == 1
+    assert step(dk=64, dv=64) == 2      # d = 128 only
+    assert step(xv=MIS) == 3
+    assert step(dt=MIS) == 3
+
+
 def test_layer_workspace_and_argument_checks(lib):
     n = ctypes.c_size_t(0)
     assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, ctypes.byref(n)) == 0

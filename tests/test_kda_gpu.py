@@ -371,3 +371,56 @@ def test_layer_zero_gate_input_halves_output(kda):
     d["o_gate_raw"] = torch.full_like(d["o_gate_raw"], 100.0)
     full, _ = run_layer(kda, d)
     torch.testing.assert_close(2 * half, full, rtol=1e-6, atol=1e-6)
+
+
+# ------------------------------------------------------------------------ layer decode (conv cache)
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_layer_decode_steps_equal_layer_over_the_same_tokens(kda, io):
+    """n layer-decode steps from an empty conv cache give the layer's outputs over those n
+    tokens and its final state; the cache ends holding the last three raw tokens, bit for bit."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    B, T, H, d = 3, 9, 4, 128
+    L = inputs.layer_inputs(B, T, H, d, d, io=ioname, seed=60, s0_std=0.05, dt_bias_std=0.4, gain_std=0.2)
+    dev = "cuda"
+    to = lambda x: None if x is None else x.contiguous().to(dev)
+    state = L["s0"].clone().to(dev)
+    caches = [torch.zeros((B, 3, H * d), dtype=io, device=dev) for _ in range(3)]
+    outs = []
+    for t in range(T):
+        o = kda.kda_layer_decode_step(
+            to(L["q_raw"][:, t]), to(L["k_raw"][:, t]), to(L["v_raw"][:, t]), to(L["conv_q"]), to(L["conv_k"]),
+            to(L["conv_v"]), *caches, to(L["g_raw"][:, t]), to(L["A_log"]), to(L["dt_bias"]), to(L["b_raw"][:, t]),
+            to(L["o_gate_raw"][:, t]), state, to(L["o_norm_w"]))
+        outs.append(o)
+    kda.kda_check_device_error()
+    out = torch.stack(outs, 1)
+    ro, rs = oracle_layer(L, io)
+    assert err(f64(out), ro, io, stored_bf16=2) <= 1.0
+    assert serr(f64(state), rs, io) <= 1.0
+    for c, n in zip(caches, ("q_raw", "k_raw", "v_raw")):
+        assert torch.equal(c.cpu(), L[n][:, T - 3:T].contiguous())
+
+
+def test_layer_decode_continues_a_layer_prefill(kda):
+    """Prefill the layer over 70 tokens, then decode 5 more with the cache seeded from the last
+    three raw tokens and the prefill's final state: the outputs equal the layer over 75 tokens."""
+    B, T0, T1, H, d = 2, 70, 5, 3, 128
+    L = inputs.layer_inputs(B, T0 + T1, H, d, d, io="bf16", seed=61, dt_bias_std=0.3)
+    dev = "cuda"
+    to = lambda x: None if x is None else x.contiguous().to(dev)
+    head = {n: (v if v is None or n in ("conv_q", "conv_k", "conv_v", "A_log", "dt_bias", "o_norm_w", "s0")
+                else v[:, :T0].contiguous()) for n, v in L.items()}
+    _, state = run_layer(kda, head)
+    caches = [to(L[n][:, T0 - 3:T0]) for n in ("q_raw", "k_raw", "v_raw")]
+    outs = []
+    for t in range(T0, T0 + T1):
+        outs.append(kda.kda_layer_decode_step(
+            to(L["q_raw"][:, t]), to(L["k_raw"][:, t]), to(L["v_raw"][:, t]), to(L["conv_q"]), to(L["conv_k"]),
+            to(L["conv_v"]), *caches, to(L["g_raw"][:, t]), to(L["A_log"]), to(L["dt_bias"]), to(L["b_raw"][:, t]),
+            to(L["o_gate_raw"][:, t]), state, to(L["o_norm_w"])))
+    kda.kda_check_device_error()
+    ro, rs = oracle_layer(L, torch.bfloat16)
+    assert err(f64(torch.stack(outs, 1)), ro[:, T0:], torch.bfloat16, stored_bf16=2) <= 1.0
+    assert serr(f64(state), rs, torch.bfloat16) <= 1.0
