@@ -54,10 +54,10 @@ def _load():
             lib.kda_oracle_decode.argtypes = [_dp] * 7 + [i] * 5
             lib.kda_oracle_short_conv_silu.argtypes = [_dp] * 3 + [i] * 5
             lib.kda_oracle_l2norm.argtypes = [_dp, _dp, sz, i, d]
-            lib.kda_oracle_gate.argtypes = [_dp] * 4 + [i] * 4
+            lib.kda_oracle_gate.argtypes = [_dp] * 3 + [d, _dp] + [i] * 4
             lib.kda_oracle_sigmoid.argtypes = [_dp, _dp, sz]
             lib.kda_oracle_out_norm_gate.argtypes = [_dp, _dp, _dp, d, i, _dp, sz, i]
-            lib.kda_oracle_layer.argtypes = [_dp] * 12 + [d, d, i, _dp, _dp, _dp] + [i] * 6
+            lib.kda_oracle_layer.argtypes = [_dp] * 9 + [d] + [_dp] * 3 + [d, d, i, _dp, _dp, _dp] + [i] * 6
             lib.kda_oracle_max_threads.restype = i
             _lib = lib
     return _lib
@@ -135,14 +135,19 @@ def l2norm(x, eps=1e-6):
     return y
 
 
-def gate(x, A_log, dt_bias=None):
-    """g = -exp(A_log[h]) * softplus(x + dt_bias[h, c]).  x: [B, T, H, dk]; A_log: [H]."""
+def gate(x, A_log, dt_bias=None, *, lower_bound=None):
+    """g = max(-exp(A_log[h]) * softplus(x + dt_bias[h, c]), lower_bound).
+
+    x: [B, T, H, dk]; A_log: [H]; lower_bound None means no bound (the Kimi-K3
+    linear-attention config's gate_lower_bound, read as a bound on the log-decay).
+    """
     x, A_log, dt_bias = _f64(x), _f64(A_log), _f64(dt_bias)
     B, T, H, dk = x.shape
     assert A_log.shape == (H,)
     assert dt_bias is None or dt_bias.size == H * dk
     g = np.zeros_like(x)
-    _load().kda_oracle_gate(_ptr(x), _ptr(A_log), _ptr(dt_bias), _ptr(g), B, T, H, dk)
+    lb = float("-inf") if lower_bound is None else float(lower_bound)
+    _load().kda_oracle_gate(_ptr(x), _ptr(A_log), _ptr(dt_bias), lb, _ptr(g), B, T, H, dk)
     return g
 
 
@@ -167,11 +172,12 @@ def out_norm_gate(o, z, gain=None, eps=1e-6, io_bf16=False):
 
 def layer(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
           o_gate_raw, o_norm_w=None, *, norm_eps=1e-6, l2_eps=1e-6, io_bf16=True,
-          s0=None, nthreads=0):
+          s0=None, gate_lower_bound=None, nthreads=0):
     """The KDA layer core: conv+SiLU, q/k L2-norm, gate, beta, recurrence, RMSNorm x sigmoid gate.
 
     q_raw, k_raw: [B, T, H*dk]; v_raw: [B, T, H*dv]; g_raw: [B, T, H, dk]; b_raw: [B, T, H];
-    o_gate_raw: [B, T, H, dv].  Returns (out [B, T, H, dv], S_T [B, H, dk, dv]).
+    o_gate_raw: [B, T, H, dv]; gate_lower_bound None = unbounded gate.
+    Returns (out [B, T, H, dv], S_T [B, H, dk, dv]).
     """
     arrs = [q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
             o_gate_raw, o_norm_w, s0]
@@ -187,7 +193,9 @@ def layer(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_
     sT = np.zeros((B, H, dk, dv))
     _load().kda_oracle_layer(
         _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
-        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
+        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias),
+        float("-inf") if gate_lower_bound is None else float(gate_lower_bound),
+        _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
         float(norm_eps), float(l2_eps), 1 if io_bf16 else 0, _ptr(s0), _ptr(out), _ptr(sT),
         B, T, H, dk, dv, nthreads,
     )

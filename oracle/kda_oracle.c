@@ -205,12 +205,14 @@ void kda_oracle_l2norm(const double *x, double *y, size_t rows, int d, double ep
     }
 }
 
-/* Per-channel log-decay gate: g = -exp(A_log[h]) * softplus(x + dt_bias[h*dk + c]).
- * x: [B, T, H, dk]; A_log: [H]; dt_bias: [H*dk] or NULL (zero).
+/* Per-channel log-decay gate: g = max(-exp(A_log[h]) * softplus(x + dt_bias[h*dk + c]), lb).
+ * x: [B, T, H, dk]; A_log: [H]; dt_bias: [H*dk] or NULL (zero); lb = -INFINITY for no bound.
  * (maxtext PR #5548 review, item 2: exp(A_log) drives the state decay, dt_bias is
- *  per channel [heads*dk], both F32.) */
-void kda_oracle_gate(const double *x, const double *A_log, const double *dt_bias, double *g,
-                     int B, int T, int H, int dk)
+ *  per channel [heads*dk], both F32.  The Kimi-K3 linear-attention config sets
+ *  gate_lower_bound = -5.0 without its formula; the plainest reading, taken here, is a
+ *  lower bound on the log-decay itself: per-token decay no stronger than exp(lb).) */
+void kda_oracle_gate(const double *x, const double *A_log, const double *dt_bias, double lb,
+                     double *g, int B, int T, int H, int dk)
 {
     const size_t n = (size_t)B * T * H;
     for (size_t r = 0; r < n; ++r) {
@@ -218,7 +220,8 @@ void kda_oracle_gate(const double *x, const double *A_log, const double *dt_bias
         const double scale = exp(A_log[h]);
         for (int c = 0; c < dk; ++c) {
             const double bias = dt_bias ? dt_bias[(size_t)h * dk + c] : 0.0;
-            g[r * dk + c] = -scale * softplus(x[r * dk + c] + bias);
+            const double v = -scale * softplus(x[r * dk + c] + bias);
+            g[r * dk + c] = v < lb ? lb : v;
         }
     }
 }
@@ -274,17 +277,18 @@ void kda_oracle_out_norm_gate(const double *o, const double *z, const double *ga
 /* The KDA layer core:
  *   q = l2norm(SiLU(conv_q * q_raw)),  k = l2norm(SiLU(conv_k * k_raw)),
  *   v = SiLU(conv_v * v_raw),
- *   g = -exp(A_log) softplus(g_raw + dt_bias),  beta = sigmoid(b_raw),
+ *   g = max(-exp(A_log) softplus(g_raw + dt_bias), lb),  beta = sigmoid(b_raw),
  *   o = gated delta rule(q, k, v, g, beta; S0) -> (o, S_T),
  *   out = out_norm_gate(o, o_gate_raw).
  * q_raw, k_raw: [B, T, H*dk]; v_raw: [B, T, H*dv]; g_raw: [B, T, H, dk];
  * b_raw: [B, T, H]; o_gate_raw: [B, T, H, dv]; conv_*: [H*d, 4]; A_log: [H];
- * dt_bias: [H*dk] or NULL; o_norm_w: [dv] or NULL; s0, sT: [B, H, dk, dv] or NULL. */
+ * dt_bias: [H*dk] or NULL; lb: the gate's lower bound (-INFINITY: none);
+ * o_norm_w: [dv] or NULL; s0, sT: [B, H, dk, dv] or NULL. */
 void kda_oracle_layer(const double *q_raw, const double *k_raw, const double *v_raw,
                       const double *conv_q, const double *conv_k, const double *conv_v,
                       const double *g_raw, const double *A_log, const double *dt_bias,
-                      const double *b_raw, const double *o_gate_raw, const double *o_norm_w,
-                      double norm_eps, double l2_eps, int io_bf16, const double *s0,
+                      double lb, const double *b_raw, const double *o_gate_raw,
+                      const double *o_norm_w, double norm_eps, double l2_eps, int io_bf16, const double *s0,
                       double *out, double *sT, int B, int T, int H, int dk, int dv,
                       int nthreads)
 {
@@ -302,7 +306,7 @@ void kda_oracle_layer(const double *q_raw, const double *k_raw, const double *v_
     kda_oracle_short_conv_silu(v_raw, conv_v, vc, B, T, H * dv, 1, nthreads);
     kda_oracle_l2norm(qc, qc, nb, dk, l2_eps);
     kda_oracle_l2norm(kc, kc, nb, dk, l2_eps);
-    kda_oracle_gate(g_raw, A_log, dt_bias, g, B, T, H, dk);
+    kda_oracle_gate(g_raw, A_log, dt_bias, lb, g, B, T, H, dk);
     kda_oracle_sigmoid(b_raw, beta, nb);
     kda_oracle_recurrent(qc, kc, vc, g, beta, s0, o, sT, B, T, H, dk, dv, 1, nthreads);
     kda_oracle_out_norm_gate(o, o_gate_raw, o_norm_w, norm_eps, io_bf16, out, nb, dv);

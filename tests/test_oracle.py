@@ -299,6 +299,24 @@ def test_gate_special_values_and_library_softplus():
     assert np.all(g < 0)
 
 
+def test_gate_lower_bound():
+    """The bound replaces exactly the log-decays below it and leaves the rest bit for bit;
+    a bound of 0 removes every decay; -inf is no bound."""
+    rng = np.random.default_rng(27)
+    B, T, H, dk = 2, 5, 3, 16
+    A = rng.uniform(0, math.log(8), H)
+    bias = rng.standard_normal(H * dk) * 0.5
+    x = rng.standard_normal((B, T, H, dk)) * 2
+    g = oracle.gate(x, A, bias)
+    gb = oracle.gate(x, A, bias, lower_bound=-5.0)
+    below = g < -5.0
+    assert 0.05 < below.mean() < 0.95   # the draw exercises both sides
+    np.testing.assert_array_equal(gb[~below], g[~below])
+    assert np.all(gb[below] == -5.0) and np.all(gb >= -5.0)
+    np.testing.assert_array_equal(oracle.gate(x, A, bias, lower_bound=float("-inf")), g)
+    assert np.all(oracle.gate(x, A, bias, lower_bound=0.0) == 0.0)
+
+
 def test_sigmoid_matches_scipy():
     x = np.linspace(-40, 40, 101)
     assert _rel(oracle.sigmoid(x), scipy.special.expit(x)) < 1e-15
@@ -324,9 +342,11 @@ def test_out_norm_gate_closed_forms():
     assert np.max(np.abs(yb - 2 * y) / np.abs(2 * y)) <= 2.0 ** -8
 
 
-def test_layer_wiring_with_identity_conv():
+@pytest.mark.parametrize("lb", [None, -1.5])
+def test_layer_wiring_with_identity_conv(lb):
     """One-hot (identity) conv taps: the layer equals the prologue built from torch library
-    ops, the recurrence, then RMSNorm x sigmoid gate built from numpy."""
+    ops, the recurrence, then RMSNorm x sigmoid gate built from numpy (with the gate's
+    lower bound, when given, applied by numpy's maximum)."""
     rng = np.random.default_rng(25)
     B, T, H, d = 2, 9, 2, 8
     q_raw = rng.standard_normal((B, T, H * d))
@@ -342,7 +362,7 @@ def test_layer_wiring_with_identity_conv():
     w = np.zeros((H * d, 4))
     w[:, 3] = 1.0
     out, sT = oracle.layer(q_raw, k_raw, v_raw, w, w, w, g_raw, A, bias, b_raw, z, gain,
-                           io_bf16=False, s0=s0)
+                           io_bf16=False, s0=s0, gate_lower_bound=lb)
     F = torch.nn.functional
     silu = lambda a: F.silu(torch.from_numpy(a)).numpy()
     qn = silu(q_raw).reshape(B, T, H, d)
@@ -352,12 +372,43 @@ def test_layer_wiring_with_identity_conv():
     vn = silu(v_raw).reshape(B, T, H, d)
     gg = -np.exp(A)[None, None, :, None] * F.softplus(
         torch.from_numpy(g_raw + bias.reshape(H, d))).numpy()
+    if lb is not None:
+        assert np.mean(gg < lb) > 0.1
+        gg = np.maximum(gg, lb)
     bb = scipy.special.expit(b_raw)
     o, s_ref = oracle.recurrent(qn, kn, vn, gg, bb, s0)
     rms = np.sqrt(np.mean(o * o, -1, keepdims=True) + 1e-6)
     ref = gain * (o / rms) * scipy.special.expit(z)
     assert _rel(out, ref) < 1e-12
     assert _rel(sT, s_ref) < 1e-12
+
+
+def test_layer_gate_bound_zero_equals_vanishing_decay_rate():
+    """A gate bound of 0 and exp(A_log) -> 0 are two routes to g = 0 (the ungated delta
+    rule); a bound below every log-decay changes nothing."""
+    rng = np.random.default_rng(28)
+    B, T, H, d = 1, 10, 2, 8
+    raw = [rng.standard_normal((B, T, H * d)) for _ in range(3)]
+    ws = [rng.standard_normal((H * d, 4)) * 0.5 for _ in range(3)]
+    g_raw = rng.standard_normal((B, T, H, d))
+    b_raw = rng.standard_normal((B, T, H))
+    z = rng.standard_normal((B, T, H, d))
+    A = rng.uniform(0, math.log(8), H)
+    s0 = rng.standard_normal((B, H, d, d)) * 0.2
+    o1, s1 = oracle.layer(*raw, *ws, g_raw, A, None, b_raw, z, None, io_bf16=False, s0=s0,
+                          gate_lower_bound=0.0)
+    o2, s2 = oracle.layer(*raw, *ws, g_raw, np.full(H, -800.0), None, b_raw, z, None,
+                          io_bf16=False, s0=s0)
+    assert _rel(o1, o2) < 1e-14 and _rel(s1, s2) < 1e-14
+    gmin = oracle.gate(g_raw, A, None).min()
+    o3, s3 = oracle.layer(*raw, *ws, g_raw, A, None, b_raw, z, None, io_bf16=False, s0=s0,
+                          gate_lower_bound=gmin - 1.0)
+    o4, s4 = oracle.layer(*raw, *ws, g_raw, A, None, b_raw, z, None, io_bf16=False, s0=s0)
+    np.testing.assert_array_equal(o3, o4)
+    np.testing.assert_array_equal(s3, s4)
+    o5, _ = oracle.layer(*raw, *ws, g_raw, A, None, b_raw, z, None, io_bf16=False, s0=s0,
+                         gate_lower_bound=-1.0)
+    assert np.max(np.abs(o5 - o4)) > 1e-3
 
 
 def test_layer_conv_is_causal_per_channel():
