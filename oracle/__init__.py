@@ -101,6 +101,36 @@ def recurrent(q, k, v, g, beta, s0=None, *, delta=True, nthreads=0):
     return o, sT
 
 
+def recurrent_varlen(q, k, v, g, beta, cu_seqlens, s0=None, *, nthreads=0):
+    """N packed sequences of different lengths, each through the token-by-token recurrence
+    from its own initial state (no state crosses a sequence boundary).
+
+    q, k, g: [T_total, H, dk]; v: [T_total, H, dv]; beta: [T_total, H]; cu_seqlens: N + 1
+    offsets (sequence n is tokens cu[n] .. cu[n+1]-1); s0: [N, H, dk, dv] or None.
+    Returns (o [T_total, H, dv], S_T [N, H, dk, dv]); o is zero at tokens no sequence covers.
+    """
+    q, k, v, g, beta, s0 = map(_f64, (q, k, v, g, beta, s0))
+    cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
+    N = len(cu) - 1
+    Tt, H, dk = q.shape
+    dv = v.shape[-1]
+    assert N >= 1 and cu[0] >= 0 and cu[-1] <= Tt and all(a <= b for a, b in zip(cu, cu[1:]))
+    assert s0 is None or s0.shape == (N, H, dk, dv)
+    o = np.zeros((Tt, H, dv))
+    sT = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        s_n = None if s0 is None else s0[n:n + 1]
+        if b == a:
+            sT[n] = 0.0 if s_n is None else s_n[0]
+            continue
+        on, sn = recurrent(q[None, a:b], k[None, a:b], v[None, a:b], g[None, a:b], beta[None, a:b],
+                           s_n, nthreads=nthreads)
+        o[a:b] = on[0]
+        sT[n] = sn[0]
+    return o, sT
+
+
 def decode(q, k, v, g, beta, state, *, nthreads=0):
     """One decode step.  q, k, g: [B, H, dk]; v: [B, H, dv]; beta: [B, H];
     state: [B, H, dk, dv].  Returns (o [B, H, dv], new_state) — the input is not modified."""

@@ -218,6 +218,51 @@ def test_empty_sequence_returns_initial_state():
     np.testing.assert_array_equal(sT, s0)
 
 
+def test_varlen_equal_lengths_equal_the_batched_call():
+    """Packed sequences of one common length give the batched result bit for bit."""
+    rng = np.random.default_rng(14)
+    B, T, H = 3, 11, 2
+    q, k, v, g, beta, s0 = _rand_inputs(rng, B, T, H, 6, 5)
+    o, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    pk = lambda x: x.reshape((B * T,) + x.shape[2:])
+    ov, sv = oracle.recurrent_varlen(pk(q), pk(k), pk(v), pk(g), pk(beta), np.arange(B + 1) * T, s0)
+    np.testing.assert_array_equal(ov, pk(o))
+    np.testing.assert_array_equal(sv, sT)
+
+
+def test_varlen_ragged_equals_chunked_form_per_sequence():
+    """Ragged lengths (0 and 1 among them): every sequence equals the chunkwise rewrite run
+    on it alone, and a zero-length sequence passes its initial state through."""
+    rng = np.random.default_rng(15)
+    lens = [5, 0, 1, 17, 9, 0, 33]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    Tt, H, dk, dv = int(cu[-1]), 2, 6, 4
+    q, k, v, g, beta, _ = _rand_inputs(rng, 1, Tt, H, dk, dv, s0_std=0)
+    s0 = rng.standard_normal((len(lens), H, dk, dv)) * 0.1
+    o, sT = oracle.recurrent_varlen(q[0], k[0], v[0], g[0], beta[0], cu, s0)
+    for n, (a, b) in enumerate(zip(cu[:-1], cu[1:])):
+        if a == b:
+            np.testing.assert_array_equal(sT[n], s0[n])
+            continue
+        oc, sc = chunked(q[:, a:b], k[:, a:b], v[:, a:b], g[:, a:b], beta[:, a:b], s0[n:n + 1], chunk=4)
+        assert _rel(o[a:b], oc[0]) < 1e-12 and _rel(sT[n], sc[0]) < 1e-12
+
+
+def test_varlen_sequences_are_isolated():
+    """Changing one sequence's tokens changes no other sequence's outputs or final state."""
+    rng = np.random.default_rng(16)
+    cu = np.array([0, 6, 13, 20])
+    q, k, v, g, beta, _ = _rand_inputs(rng, 1, 20, 2, 5, 5, s0_std=0)
+    o1, s1 = oracle.recurrent_varlen(q[0], k[0], v[0], g[0], beta[0], cu)
+    v2 = v.copy()
+    v2[0, 6:13] += 1.0
+    o2, s2 = oracle.recurrent_varlen(q[0], k[0], v2[0], g[0], beta[0], cu)
+    np.testing.assert_array_equal(o1[:6], o2[:6])
+    np.testing.assert_array_equal(o1[13:], o2[13:])
+    np.testing.assert_array_equal(s1[[0, 2]], s2[[0, 2]])
+    assert np.max(np.abs(o1[6:13] - o2[6:13])) > 1e-3
+
+
 def test_state_norm_bound():
     """||k|| = 1, beta in [0, 1], g <= 0  =>  ||S_t||_2 <= ||S_{t-1}||_2 + beta_t ||v_t||."""
     rng = np.random.default_rng(13)
