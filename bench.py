@@ -38,6 +38,7 @@ METRIC = "KDA tokens/s (prefill, H=96 d=128) and decode GB/s; fraction of roofli
 PREFILL = "prefill_bf16_B4_T8192_H96_d128"
 DECODE = "decode_bf16_B256_H96_d128_x20"
 LAYER = "layer_bf16_B2_T16384_H96_d128"
+VARLEN = "varlen_bf16_T32768_H96_d128"
 L2_BYTES = 126 * 1024 * 1024
 
 # Algorithmic work (per token-head, d = 128, C = 64):
@@ -59,7 +60,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--skip", default="", help="comma list of: decode,layer_decode,layer,e2e,cpu")
+    ap.add_argument("--skip", default="", help="comma list of: varlen,decode,layer_decode,layer,e2e,cpu")
     return ap.parse_args()
 
 
@@ -285,6 +286,38 @@ def run_ours(args):
     del dv_in, out, sT, d
     torch.cuda.empty_cache()
 
+    # ------------------------------------------------------------------ packed variable length
+    if "varlen" not in skip:
+        wv = inputs.WORKLOADS[VARLEN]
+        lens = inputs.packed_lengths(wv["total"], wv["max_len"], wv["seed"])
+        dl = inputs.varlen_inputs(lens, wv["H"], wv["dk"], wv["dv"], io=wv["io"], seed=wv["seed"])
+        xv = {n: dl[n].to(dev) for n in ("q", "k", "v", "g", "beta", "cu_seqlens")}
+        Tt, Hv, Nv = wv["total"], wv["H"], len(lens)
+        ov = torch.empty((Tt, Hv, wv["dv"]), dtype=torch.bfloat16, device=dev)
+        sv = torch.empty((Nv, Hv, wv["dk"], wv["dv"]), dtype=torch.float32, device=dev)
+
+        def varlen_step():
+            kda.kda_forward_chunked_varlen(xv["q"], xv["k"], xv["v"], xv["g"], xv["beta"], xv["cu_seqlens"],
+                                           None, ov, sv, stream=stream)
+
+        total_v, per_v = timed(torch, varlen_step, args.steps, args.warmup, stream, barrier)
+        kda.kda_check_device_error(stream)
+        ms_v = max_over_ranks(total_v / args.steps)
+        lms_v = max_over_ranks(statistics.mean(per_v))
+        bytes_v = Tt * Hv * PREFILL_BYTES_PER_TOKEN_HEAD + Nv * Hv * wv["dk"] * wv["dv"] * 4
+        ach_v = bytes_v / (lms_v / 1e3) / 1e9
+        res["varlen"] = {
+            "workload": f"kda_forward_chunked_varlen, {Tt} tokens packed as {Nv} sequences of "
+                        f"{min(lens)}..{max(lens)} tokens (uniform 1..{wv['max_len']}, seed {wv['seed']}), "
+                        f"H={Hv} dk=dv=128 bf16, zero initial state",
+            "value": round(aggregate_rate(Tt, ms_v, ws), 1), "unit": "tokens/s", "ms_per_step": round(ms_v, 4),
+            "roofline": {"bound": "hbm", "achieved": round(ach_v, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach_v / pk["hbm_gbs"], 4), "traffic": traffic_for("kda_chunk_tc"),
+                         "kernel": "kda_chunk_tc", "launch_ms": round(lms_v, 4), "bytes_per_launch": bytes_v}}
+        launches_per["varlen"] = 1
+        del xv, ov, sv, dl
+        torch.cuda.empty_cache()
+
     # ------------------------------------------------------------------ decode
     if "decode" not in skip:
         wd = inputs.WORKLOADS[DECODE]
@@ -403,8 +436,8 @@ def run_ours(args):
     if rank == 0 and ws == 1 and "cpu" not in skip:
         cpu = cpu_baseline_prefill()
 
-    gpu_launches = args.steps * launches_per["prefill"] + launches_per.get("decode", 0) + \
-        launches_per.get("layer_decode", 0) + launches_per.get("layer", 0)
+    gpu_launches = args.steps * (launches_per["prefill"] + launches_per.get("varlen", 0)) + \
+        launches_per.get("decode", 0) + launches_per.get("layer_decode", 0) + launches_per.get("layer", 0)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

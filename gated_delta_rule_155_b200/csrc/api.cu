@@ -92,7 +92,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_abi_version(void) { return 100; }
+int kda_abi_version(void) { return 101; }
 
 kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *initial_state, void *out,
@@ -111,6 +111,32 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
                                                           (size_t)B * H * dk * dv, s));
     kda::ChunkArgs a{q, k, v, g, beta, initial_state, out, final_state, B, T, H, dk, dv,
                      io_of(io), false, false, false, false, error_word()};
+    if (kda::chunk_tc_supported(a)) return cuda_status(kda::launch_chunk_tc(a, s));
+    if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
+    return cuda_status(kda::launch_chunk_simt(a, s));
+}
+
+kda_status_t kda_forward_chunked_varlen(const void *q, const void *k, const void *v, const void *g,
+                                        const void *beta, const float *initial_state, void *out,
+                                        float *final_state, const int *cu_seqlens, int N,
+                                        int T_total, int H, int dk, int dv, int chunk,
+                                        kda_dtype_t io, kda_stream_t stream)
+{
+    kda_status_t st = check_dims(N, T_total, H, dk, dv, io);
+    if (st != KDA_OK) return st;
+    if ((long long)N * H > INT32_MAX / 2) return KDA_ERR_UNSUPPORTED;
+    if (chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (T_total > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, initial_state, out, final_state, cu_seqlens};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T_total == 0) return cuda_status(kda::launch_fill_state(initial_state, final_state,
+                                                                (size_t)N * H * dk * dv, s));
+    // the kernels take B = N sequences over a token axis of T = T_total rows
+    kda::ChunkArgs a{q, k, v, g, beta, initial_state, out, final_state, N, T_total, H, dk, dv,
+                     io_of(io), false, false, false, false, error_word(), cu_seqlens};
     if (kda::chunk_tc_supported(a)) return cuda_status(kda::launch_chunk_tc(a, s));
     if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
     return cuda_status(kda::launch_chunk_simt(a, s));
@@ -143,15 +169,15 @@ kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_d
 kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void *v_raw,
                                const float *conv_q, const float *conv_k, const float *conv_v,
                                const void *g_raw, const float *A_log, const float *dt_bias,
-                               const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
-                               float norm_eps, const float *initial_state, void *out,
-                               float *final_state, void *workspace, size_t workspace_bytes,
+                               float gate_lower_bound, const void *b_raw, const void *o_gate_raw,
+                               const float *o_norm_w, float norm_eps, const float *initial_state,
+                               void *out, float *final_state, void *workspace, size_t workspace_bytes,
                                int B, int T, int H, int dk, int dv, kda_dtype_t io,
                                kda_stream_t stream)
 {
     kda_status_t st = check_dims(B, T, H, dk, dv, io);
     if (st != KDA_OK) return st;
-    if (!(norm_eps >= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (!(norm_eps >= 0.0f) || !(gate_lower_bound <= 0.0f)) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !g_raw ||
                   !A_log || !b_raw || !o_gate_raw || !out))
         return KDA_ERR_INVALID_ARG;
@@ -170,7 +196,7 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
     float *wg = (float *)(ws + w.g), *wb = (float *)(ws + w.beta), *wo = (float *)(ws + w.o);
 
     kda::PrologueArgs pa{q_raw, k_raw, v_raw, g_raw, b_raw, conv_q, conv_k, conv_v, A_log, dt_bias,
-                         wq, wk, wv, wg, wb, B, T, H, dk, dv, io_of(io)};
+                         gate_lower_bound, wq, wk, wv, wg, wb, B, T, H, dk, dv, io_of(io)};
     cudaError_t e = kda::launch_prologue(pa, s);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     kda::ChunkArgs ca{wq, wk, wv, wg, wb, initial_state, wo, final_state, B, T, H, dk, dv,
@@ -184,15 +210,15 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
 kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const void *v_raw,
                                    const float *conv_q, const float *conv_k, const float *conv_v,
                                    void *cache_q, void *cache_k, void *cache_v, const void *g_raw,
-                                   const float *A_log, const float *dt_bias, const void *b_raw,
-                                   const void *o_gate_raw, const float *o_norm_w, float norm_eps,
-                                   float *state, void *out, int B, int H, int dk, int dv,
+                                   const float *A_log, const float *dt_bias, float gate_lower_bound,
+                                   const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
+                                   float norm_eps, float *state, void *out, int B, int H, int dk, int dv,
                                    kda_dtype_t io, kda_stream_t stream)
 {
     kda_status_t st = check_dims(B, 1, H, dk, dv, io);
     if (st != KDA_OK) return st;
     if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
-    if (!(norm_eps >= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (!(norm_eps >= 0.0f) || !(gate_lower_bound <= 0.0f)) return KDA_ERR_INVALID_ARG;
     if (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !cache_q || !cache_k || !cache_v ||
         !g_raw || !A_log || !b_raw || !o_gate_raw || !state || !out)
         return KDA_ERR_INVALID_ARG;
@@ -201,8 +227,8 @@ kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const v
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
     kda::LayerDecodeArgs a{q_raw, k_raw, v_raw, cache_q, cache_k, cache_v, conv_q, conv_k, conv_v,
-                           g_raw, A_log, dt_bias, b_raw, o_gate_raw, o_norm_w, norm_eps, state, out,
-                           B, H, io_of(io)};
+                           g_raw, A_log, dt_bias, gate_lower_bound, b_raw, o_gate_raw, o_norm_w,
+                           norm_eps, state, out, B, H, io_of(io)};
     return cuda_status(kda::launch_layer_decode(a, (cudaStream_t)stream));
 }
 

@@ -88,7 +88,7 @@ KDA_DEVICE void axpy4(float4 &acc, float4 a, float4 r0, float4 r1, float4 r2, fl
 __global__ void __launch_bounds__(FNT, 1)
 kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, const float *__restrict__ v,
                      const float *__restrict__ g, const float *__restrict__ beta, const float *__restrict__ s0,
-                     float *__restrict__ out, float *__restrict__ sT, int T, int H)
+                     float *__restrict__ out, float *__restrict__ sT, int Ttot, int H, const int *__restrict__ cu)
 {
     extern __shared__ __align__(16) float fsm[];
     float *XQ = fsm + F_XQ, *XK = fsm + F_XK, *XT = fsm + F_XT, *Vs = fsm + F_V, *Ss = fsm + F_S;
@@ -100,6 +100,8 @@ kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, c
     const int tid = threadIdx.x;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int vh = blockIdx.y;   // value half
+    const SeqSpan span = seq_span(cu, b, Ttot);   // this sequence's rows row0 .. row0 + T - 1
+    const int T = span.len, row0 = span.row0;
     const size_t soff = (size_t)bh * FD * FD + (size_t)vh * FDH;
 
     if (tid < FD) ONE[tid] = F32_INV_SC;
@@ -119,7 +121,7 @@ kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, c
         for (int idx = tid; idx < FC * FD / 4; idx += FNT) {
             const int i = idx >> 5, c4 = (idx & 31) * 4;
             const bool ok = t0 + i < T;
-            const size_t off = ok ? ((size_t)(b * T + t0 + i) * H + h) * FD + c4 : 0;
+            const size_t off = ok ? ((size_t)(row0 + t0 + i) * H + h) * FD + c4 : 0;
             cp_async16(XQ + i * LDX + c4, q + off, ok);
             cp_async16(XK + i * LDX + c4, k + off, ok);
             cp_async16(XT + i * LDX + c4, g + off, ok);
@@ -127,10 +129,10 @@ kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, c
         for (int idx = tid; idx < FC * FDH / 4; idx += FNT) {
             const int i = idx >> 4, j4 = (idx & 15) * 4;
             const bool ok = t0 + i < T;
-            const size_t off = ok ? ((size_t)(b * T + t0 + i) * H + h) * FD + vh * FDH + j4 : 0;
+            const size_t off = ok ? ((size_t)(row0 + t0 + i) * H + h) * FD + vh * FDH + j4 : 0;
             cp_async16(Vs + i * LDH + j4, v + off, ok);
         }
-        if (tid < FC) BETAs[tid] = t0 + tid < T ? beta[(size_t)(b * T + t0 + tid) * H + h] : 0.0f;
+        if (tid < FC) BETAs[tid] = t0 + tid < T ? beta[(size_t)(row0 + t0 + tid) * H + h] : 0.0f;
         tc::cp_async_commit();
         tc::cp_async_wait_all();
         __syncthreads();
@@ -268,12 +270,12 @@ kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, c
                     for (int wd = 0; wd < 4; ++wd) {
                         for (uint32_t mk = MASK[I * 4 + wd]; mk != 0u; mk &= mk - 1u) {
                             const int c = 32 * wd + __ffs((int)mk) - 1;
-                            const size_t ri = ((size_t)(b * T + t0 + i) * H + h) * FD + c;
+                            const size_t ri = ((size_t)(row0 + t0 + i) * H + h) * FD + c;
                             const float qi = vi ? q[ri] : 0.0f, ki = vi ? k[ri] : 0.0f;
                             float w = 1.0f;   // exp(G_i - G_j), built backwards from j = i
                             for (int j = i; j >= 16 * I; --j) {
                                 const bool vj = t0 + j < T;
-                                const size_t rj = ((size_t)(b * T + t0 + j) * H + h) * FD + c;
+                                const size_t rj = ((size_t)(row0 + t0 + j) * H + h) * FD + c;
                                 const float kj = vj ? k[rj] : 0.0f;
                                 Ps[i * LDH + j] += qi * kj * w;
                                 if (j < i) As[i * LDH + j] += bi * ki * kj * w;
@@ -404,7 +406,7 @@ kda_chunk_f32_kernel(const float *__restrict__ q, const float *__restrict__ k, c
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
                 const int i = 4 * ti + a;
-                if (t0 + i < T) st4s(out + ((size_t)(b * T + t0 + i) * H + h) * FD + vh * FDH + 4 * tj, acc[a]);
+                if (t0 + i < T) st4s(out + ((size_t)(row0 + t0 + i) * H + h) * FD + vh * FDH + 4 * tj, acc[a]);
             }
         }
         __syncthreads();
@@ -465,7 +467,7 @@ cudaError_t launch_chunk_f32(const ChunkArgs &a, cudaStream_t s)
     dim3 grid((unsigned)(a.B * a.H), 2u);
     kda_chunk_f32_kernel<<<grid, FNT, F32_SMEM, s>>>((const float *)a.q, (const float *)a.k, (const float *)a.v,
                                                      (const float *)a.g, (const float *)a.beta, a.s0,
-                                                     (float *)a.out, a.sT, a.T, a.H);
+                                                     (float *)a.out, a.sT, a.T, a.H, a.cu);
     return cudaGetLastError();
 }
 

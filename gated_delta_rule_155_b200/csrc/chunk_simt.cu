@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
 kda_chunk_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const TI *__restrict__ v,
                       const TG *__restrict__ g, const TB *__restrict__ beta,
                       const float *__restrict__ s0, TO *__restrict__ out, float *__restrict__ sT,
-                      int T, int H, int dv)
+                      int Ttot, int H, int dv, const int *__restrict__ cu)
 {
     using L = SimtSmem<DK>;
     extern __shared__ float smem[];
@@ -60,6 +60,8 @@ kda_chunk_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const 
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
     const int v0 = blockIdx.y * CS_DVS;
+    const SeqSpan span = seq_span(cu, b, Ttot);   // this sequence's rows row0 .. row0 + T - 1
+    const int T = span.len, row0 = span.row0;
     const size_t state_off = (size_t)bh * DK * dv + v0;
 
     // initial state slice
@@ -79,7 +81,7 @@ kda_chunk_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const 
             float fq[4] = {0.f, 0.f, 0.f, 0.f}, fk[4] = {0.f, 0.f, 0.f, 0.f},
                   fg[4] = {0.f, 0.f, 0.f, 0.f};
             if (i < nt) {
-                const size_t off = ((size_t)(b * T + t0 + i) * H + h) * DK + c;
+                const size_t off = ((size_t)(row0 + t0 + i) * H + h) * DK + c;
                 ld4(q + off, fq);
                 ld4(k + off, fk);
                 ld4(g + off, fg);
@@ -94,11 +96,11 @@ kda_chunk_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const 
         for (int idx = tid; idx < CS_C * CS_DVS / 4; idx += CS_THREADS) {
             const int i = idx / (CS_DVS / 4), j = (idx % (CS_DVS / 4)) * 4;
             float fv[4] = {0.f, 0.f, 0.f, 0.f};
-            if (i < nt) ld4(v + ((size_t)(b * T + t0 + i) * H + h) * dv + v0 + j, fv);
+            if (i < nt) ld4(v + ((size_t)(row0 + t0 + i) * H + h) * dv + v0 + j, fv);
 #pragma unroll
             for (int e = 0; e < 4; ++e) Us[i * L::LDV + j + e] = fv[e];
         }
-        if (tid < CS_C) Bs[tid] = tid < nt ? to_f32(beta[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
+        if (tid < CS_C) Bs[tid] = tid < nt ? to_f32(beta[(size_t)(row0 + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         // ---------------------------------------------------------------- G = cumsum(g)
         if (tid < DK) {
@@ -183,7 +185,7 @@ kda_chunk_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k, const 
                 for (int vv = 0; vv < 16; ++vv) o[vv] += pij * Us[j * L::LDV + part + 4 * vv];
             }
             if (i < nt) {
-                TO *orow = out + ((size_t)(b * T + t0 + i) * H + h) * dv + v0;
+                TO *orow = out + ((size_t)(row0 + t0 + i) * H + h) * dv + v0;
 #pragma unroll
                 for (int vv = 0; vv < 16; ++vv) orow[part + 4 * vv] = from_f32<TO>(o[vv]);
             }
@@ -227,7 +229,7 @@ cudaError_t launch_t(const ChunkArgs &a, cudaStream_t s)
     dim3 grid((unsigned)(a.B * a.H), (unsigned)(a.dv / CS_DVS));
     kern<<<grid, CS_THREADS, bytes, s>>>((const TI *)a.q, (const TI *)a.k, (const TI *)a.v,
                                           (const TG *)a.g, (const TB *)a.beta, a.s0, (TO *)a.out,
-                                          a.sT, a.T, a.H, a.dv);
+                                          a.sT, a.T, a.H, a.dv, a.cu);
     return cudaGetLastError();
 }
 

@@ -126,6 +126,7 @@ struct TcParams {
     float *sT;
     int T, H;
     int *err;
+    const int *cu;   // packed variable length: sequence offsets (null: fixed length T)
 };
 
 KDA_DEVICE void unpack8(const uint4 &u, float (&f)[8])
@@ -139,6 +140,10 @@ KDA_DEVICE uint4 pack8(const float (&f)[8])
                       pack_bf16x2(f[6], f[7]));
 }
 
+// PACKED: N sequences of different lengths back to back (offsets p.cu), one batch row of the
+// tensor maps; otherwise B sequences of T tokens.  The fixed-length instance carries none of
+// the packed bookkeeping.
+template <bool PACKED>
 __global__ void __launch_bounds__(NT, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -164,7 +169,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
-    const int T = p.T;
+    // this sequence's tokens: rows row0 .. row0 + T - 1 of the flattened token axis; the 4-D
+    // tensor maps address them as (token tt0 + t, batch tb)
+    const SeqSpan span = PACKED ? seq_span(p.cu, b, p.T) : SeqSpan{b * p.T, p.T};
+    const int T = span.len, row0 = span.row0;
+    const int tt0 = PACKED ? row0 : 0, tb = PACKED ? 0 : b;
     const int nchunks = (T + CK - 1) / CK;
     // a warp reaches TMEM lanes 32 (warp & 3) .. + 31; the four warps of a lane quarter split
     // the columns of every TMEM tile they read or write into column groups cg = warp >> 2
@@ -195,13 +204,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto issue_tma = [&](int n) {
         const int r = n & 1;
         uint8_t *st = sm + (r ? OFF_REG1 : OFF_REG0);
-        const int t0 = n * CK;
+        const int t0 = tt0 + n * CK;
         mbar_arrive_expect_tx(&bar_tma[r], 4 * 16384);
         for (int cb = 0; cb < 2; ++cb) {
-            tma_load_4d(st + ST_Q + cb * 8192, &tm_q, cb * 64, h, t0, b, &bar_tma[r]);
-            tma_load_4d(st + ST_K + cb * 8192, &tm_k, cb * 64, h, t0, b, &bar_tma[r]);
-            tma_load_4d(st + ST_V + cb * 8192, &tm_v, cb * 64, h, t0, b, &bar_tma[r]);
-            tma_load_4d(st + ST_G + cb * 8192, &tm_g, cb * 64, h, t0, b, &bar_tma[r]);
+            tma_load_4d(st + ST_Q + cb * 8192, &tm_q, cb * 64, h, t0, tb, &bar_tma[r]);
+            tma_load_4d(st + ST_K + cb * 8192, &tm_k, cb * 64, h, t0, tb, &bar_tma[r]);
+            tma_load_4d(st + ST_V + cb * 8192, &tm_v, cb * 64, h, t0, tb, &bar_tma[r]);
+            tma_load_4d(st + ST_G + cb * 8192, &tm_g, cb * 64, h, t0, tb, &bar_tma[r]);
         }
     };
     if (tid == 0 && nchunks > 0) issue_tma(0);
@@ -241,7 +250,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const void *src = p.beta;
         uint32_t bytes = 0;
         if (t < T) {
-            const uintptr_t ea = (uintptr_t)(p.beta + (size_t)(b * T + t) * p.H + h);
+            const uintptr_t ea = (uintptr_t)(p.beta + (size_t)(row0 + t) * p.H + h);
             bytes = (ea & 2) ? 4u : 2u;
             src = (const void *)(ea & ~(uintptr_t)3);
         }
@@ -263,7 +272,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             cp_async_wait_all();
             const int t = t0 + tid;
             const uint32_t wv = BRAW[(n & 1) * CK + tid];
-            const bool hi = t < T && (((uintptr_t)(p.beta + (size_t)(b * T + t) * p.H + h)) & 2);
+            const bool hi = t < T && (((uintptr_t)(p.beta + (size_t)(row0 + t) * p.H + h)) & 2);
             BETAsm[tid] = __uint_as_float(hi ? (wv & 0xffff0000u) : (wv << 16));
             if (n + 1 < nchunks) beta_async(n + 1);
         }
@@ -285,6 +294,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
             f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
         };
+        // Rows at or past the end of a packed sequence (the next sequence's tokens) enter as
+        // g = 0 and k = 0: they then add nothing to the decays, A, P's columns, Y or the state
+        // update, and their own output rows are not stored.  (Fixed length: the tensor maps'
+        // zero fill past T does the same.)
+        const int nvalid = T - t0;
+        const bool tail = PACKED && nvalid < CK;   // the same for the whole block
         // pass A: in-half inclusive prefix of g by an 8-lane scan; the last lane of each half
         // publishes the half-block sums
         float Gh[2][8];
@@ -293,6 +308,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int B = s == 0 ? pr : 3 - pr;
             const int i = 16 * B + 8 * th + pp;
             unpack8(*(const uint4 *)(stg + ST_G + cb * 8192 + swz(i, a)), Gh[s]);
+            if (tail && i >= nvalid) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Gh[s][e] = 0.0f;
+            }
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 float l = Gh[s][e];
@@ -374,6 +393,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float qf[8], kf[8], o[8], E1[8], E2[8], f[8];
                 unpack8(*(const uint4 *)(stg + ST_Q + off), qf);
                 unpack8(*(const uint4 *)(stg + ST_K + off), kf);
+                if (tail && i >= nvalid) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) kf[e] = 0.0f;
+                }
                 // exact diagonal of P: partial q_i . k_i over this lane's 8 channels, summed over
                 // the quarter's 4 lanes
                 float pd = 0.0f;
@@ -557,12 +580,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int wd = 0; wd < 4; ++wd) {
                 for (uint32_t mk = bmask[wd]; mk != 0u; mk &= mk - 1u) {
                     const int c = 32 * wd + __ffs((int)mk) - 1;
-                    const size_t rowi = ((size_t)(b * T + t0 + i) * p.H + h) * DD + c;
+                    const size_t rowi = ((size_t)(row0 + t0 + i) * p.H + h) * DD + c;
                     const float xi = (t0 + i < T) ? __bfloat162float((is_q ? p.q : p.k)[rowi]) : 0.0f;
                     float w = 1.0f;   // exp(G_i - G_j), built backwards from j = i
                     for (int j = i; j >= 16 * I; --j) {
                         const bool valid = t0 + j < T;
-                        const size_t rowj = ((size_t)(b * T + t0 + j) * p.H + h) * DD + c;
+                        const size_t rowj = ((size_t)(row0 + t0 + j) * p.H + h) * DD + c;
                         if (j < i && ((j >> 3) & 3) == cg) {
                             const float d = xi * (valid ? __bfloat162float(p.k[rowj]) : 0.0f) * w;
                             if (is_q) {
@@ -834,9 +857,18 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&tm_o, stg + ST_V, 0, h, t0, b);
-            tma_store_4d(&tm_o, stg + ST_V + 8192, 64, h, t0, b);
+        if (tail) {
+            // the last chunk of a packed sequence: its tile's later rows are the next
+            // sequence's, so only the valid rows are written, 16 bytes per thread and pass
+            for (int u = tid; u < CK * 16; u += NT) {
+                const int i = u >> 4, j = u & 15;
+                if (i < nvalid)
+                    *(uint4 *)(p.out + ((size_t)(row0 + t0 + i) * p.H + h) * DD + 8 * j) =
+                        *(const uint4 *)(stg + ST_V + (j >> 3) * 8192 + swz(i, j & 7));
+            }
+        } else if (tid == 0) {
+            tma_store_4d(&tm_o, stg + ST_V, 0, h, tt0 + t0, tb);
+            tma_store_4d(&tm_o, stg + ST_V + 8192, 64, h, tt0 + t0, tb);
             bulk_commit();
         }
     }
@@ -920,19 +952,25 @@ bool chunk_tc_supported(const ChunkArgs &a)
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
 {
     CUtensorMap mq, mk, mv, mg, mo;
-    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
-        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mg, a.g, a.B, a.T, a.H) ||
-        !make_map(&mo, a.out, a.B, a.T, a.H))
+    const int mb = a.cu ? 1 : a.B;   // packed sequences: one batch row of all tokens
+    if (!make_map(&mq, a.q, mb, a.T, a.H) || !make_map(&mk, a.k, mb, a.T, a.H) ||
+        !make_map(&mv, a.v, mb, a.T, a.H) || !make_map(&mg, a.g, mb, a.T, a.H) ||
+        !make_map(&mo, a.out, mb, a.T, a.H))
         return cudaErrorInvalidValue;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        attr_err = cudaFuncSetAttribute(kda_chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(kda_chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
     TcParams p{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
-               (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err};
-    kda_chunk_tc_kernel<<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
+               (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err, a.cu};
+    if (a.cu) kda_chunk_tc_kernel<true><<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
+    else kda_chunk_tc_kernel<false><<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();
 }
 

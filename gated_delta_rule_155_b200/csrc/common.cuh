@@ -55,6 +55,21 @@ KDA_DEVICE float siluf_(float x) { return x / (1.0f + __expf(-x)); }
 // log(1 + e^x) without overflow
 KDA_DEVICE float softplusf_(float x) { return x > 0.0f ? x + log1pf(__expf(-x)) : log1pf(__expf(x)); }
 
+// The tokens of sequence b: rows row0 .. row0 + len - 1 of the flattened [tokens, H, d]
+// tensors.  Fixed length (cu == nullptr): row0 = b T, len = T.  Packed variable length:
+// row0 = cu[b], len = cu[b + 1] - cu[b], both clamped into [0, T] (T = total tokens), so
+// that no access leaves the buffers whatever the offsets hold.
+struct SeqSpan {
+    int row0, len;
+};
+KDA_DEVICE SeqSpan seq_span(const int *cu, int b, int T)
+{
+    if (!cu) return SeqSpan{b * T, T};
+    const int s = min(max(cu[b], 0), T);
+    const int e = min(max(cu[b + 1], s), T);
+    return SeqSpan{s, e - s};
+}
+
 KDA_DEVICE float warp_sum(float v)
 {
 #pragma unroll

@@ -21,6 +21,7 @@ struct ChunkArgs {
     IoType io;
     bool qkv_f32, g_f32, beta_f32, out_f32;
     int *err;
+    const int *cu = nullptr;  // packed variable length: sequence offsets [B + 1], device; T = total tokens
 };
 
 struct DecodeArgs {
@@ -34,6 +35,7 @@ struct DecodeArgs {
 struct PrologueArgs {
     const void *q_raw, *k_raw, *v_raw, *g_raw, *b_raw;
     const float *conv_q, *conv_k, *conv_v, *A_log, *dt_bias;
+    float g_lb;                   // lower bound on the log-decay g (-inf: none)
     float *q, *k, *v, *g, *beta;  // workspace outputs, fp32
     int B, T, H, dk, dv;
     IoType io;
@@ -56,6 +58,7 @@ struct LayerDecodeArgs {
     const float *conv_q, *conv_k, *conv_v;  // [H*128, 4]
     const void *g_raw;                      // [B, H, 128], io
     const float *A_log, *dt_bias;           // [H]; [H*128] or null
+    float g_lb;                             // lower bound on the log-decay g (-inf: none)
     const void *b_raw, *o_gate_raw;         // [B, H]; [B, H, 128], io
     const float *gain;                      // [128] or null
     float eps;

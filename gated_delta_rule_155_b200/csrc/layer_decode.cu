@@ -4,7 +4,7 @@
 //   y_X[c] = SiLU(w_X[c,0] x[t-3,c] + w_X[c,1] x[t-2,c] + w_X[c,2] x[t-1,c] + w_X[c,3] x[t,c])
 //            for X = q, k, v, with x[t-3..t-1] taken from the conv cache, which then shifts in x[t]
 //   q^ = y_q / sqrt(|y_q|^2 + 1e-6),  k^ likewise,  v = y_v
-//   g = -exp(A_log[h]) softplus(g_raw + dt_bias),  beta = sigmoid(b_raw)
+//   g = max(-exp(A_log[h]) softplus(g_raw + dt_bias), lb),  beta = sigmoid(b_raw)
 //   S' = Diag(exp g) S;  u = beta (v - S'^T k^);  S <- S' + k^ u^T;  o = S^T q^
 //   out = gain * cast_io(o * rsqrt(mean(o^2) + eps)) * sigmoid(o_gate_raw)
 // — the same steps as the prefill path (prologue, recurrence, epilogue: the short-conv and
@@ -78,11 +78,11 @@ kda_layer_decode_kernel(LayerDecodeArgs a)
             if (lane == 0) s_part[X][warp & 3] = ss;
         }
     } else if (tid < 3 * LD_D + LD_D) {
-        // gate g = -exp(A_log[h]) softplus(g_raw + dt_bias) for channel c; alpha = exp(g)
+        // gate g = max(-exp(A_log[h]) softplus(g_raw + dt_bias), lb) for channel c; alpha = exp(g)
         const int c = tid - 3 * LD_D;
         const float bias = a.dt_bias ? a.dt_bias[(size_t)h * LD_D + c] : 0.0f;
         const float x = to_f32(((const IO *)a.g_raw)[(size_t)bh * LD_D + c]);
-        s_alpha[c] = __expf(-__expf(a.A_log[h]) * softplusf_(x + bias));
+        s_alpha[c] = __expf(fmaxf(-__expf(a.A_log[h]) * softplusf_(x + bias), a.g_lb));
         if (c == 0) s_beta = sigmoidf_(to_f32(((const IO *)a.b_raw)[bh]));
     }
     __syncthreads();

@@ -6,7 +6,8 @@
 //     y[t, c] = sum_{i=0..3} w[c, i] x[t - 3 + i, c]
 //     (open-model-atlas "Kimi-K3" linear_attn_config: short_conv_kernel_size 4;
 //      maxtext PR #5548 review item 2: {q,k,v}_conv1d.weight [heads*d, 1, 4] in F32)
-//   g = -exp(A_log[h]) softplus(g_raw + dt_bias[h, c]),  beta = sigmoid(b_raw)
+//   g = max(-exp(A_log[h]) softplus(g_raw + dt_bias[h, c]), lb),  beta = sigmoid(b_raw)
+//     (lb: the linear-attention config's gate_lower_bound, read as a bound on g itself)
 //     (maxtext PR #5548 review item 2: exp(A_log) drives the state decay)
 // Epilogue, per (b, t, h) row of dv values (one warp each):
 //   out = gain * cast_io(o * rsqrt(mean(o^2) + eps)) * sigmoid(z)
@@ -119,7 +120,7 @@ kda_prologue_kernel(PrologueArgs a)
                               a.k + (bt0 * a.H + h) * DK, rsk, t0, nt, lane);
     conv_stream<IO, DV, false>((const IO *)a.v_raw + bt0 * rsv + (size_t)h * DV, rsv, a.conv_v + (size_t)h * DV * 4,
                                a.v + (bt0 * a.H + h) * DV, rsv, t0, nt, lane);
-    // gate g = -exp(A_log[h]) softplus(g_raw + dt_bias[h, c]) and beta = sigmoid(b_raw)
+    // gate g = max(-exp(A_log[h]) softplus(g_raw + dt_bias[h, c]), lb) and beta = sigmoid(b_raw)
     {
         constexpr int N = DK / 32;
         const int c0 = N * lane;
@@ -132,7 +133,7 @@ kda_prologue_kernel(PrologueArgs a)
             float x[N];
             ldn<N>((const IO *)a.g_raw + row, x);
 #pragma unroll
-            for (int e = 0; e < N; ++e) x[e] = -scale * softplusf_(x[e] + bias[e]);
+            for (int e = 0; e < N; ++e) x[e] = fmaxf(-scale * softplusf_(x[e] + bias[e]), a.g_lb);
             stn<N>(a.g + row, x);
         }
         if (lane < nt) {

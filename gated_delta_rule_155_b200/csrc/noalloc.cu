@@ -48,7 +48,8 @@ void *scratch_on_current_device()
 
 extern "C" kda_status_t kda_layer_forward_noalloc(
     const void *q_raw, const void *k_raw, const void *v_raw, const float *conv_q, const float *conv_k,
-    const float *conv_v, const void *g_raw, const float *A_log, const float *dt_bias, const void *b_raw,
+    const float *conv_v, const void *g_raw, const float *A_log, const float *dt_bias, float gate_lower_bound,
+    const void *b_raw,
     const void *o_gate_raw, const float *o_norm_w, float norm_eps, const float *initial_state, void *out,
     float *final_state, int B, int T, int H, int dk, int dv, kda_dtype_t io, kda_stream_t stream)
 {
@@ -61,7 +62,8 @@ extern "C" kda_status_t kda_layer_forward_noalloc(
         scratch = scratch_on_current_device();
         if (!scratch) return KDA_ERR_CUDA;
     }
-    return kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
+    return kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,
+                             gate_lower_bound, b_raw,
                              o_gate_raw, o_norm_w, norm_eps, initial_state, out, final_state, scratch,
                              need > 0 ? KDA_NOALLOC_SCRATCH_BYTES : 0, B, T, H, dk, dv, io, stream);
 }

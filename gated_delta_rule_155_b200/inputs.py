@@ -161,7 +161,29 @@ def layer_inputs(B, T, H, dk, dv, *, io="bf16", seed=4, conv_std=0.5, s0_std=0.0
             "b_raw": b_raw, "o_gate_raw": o_gate, "o_norm_w": gain, "s0": s0}
 
 
-# The five workloads, by what they are.
+def packed_lengths(total: int, max_len: int, seed: int) -> list:
+    """Sequence lengths for a packed batch of `total` tokens: uniform draws in [1, max_len]
+    until the sum reaches `total`, the last one trimmed to fit."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x5E9]))
+    lens = []
+    while sum(lens) < total:
+        lens.append(int(min(rng.integers(1, max_len + 1), total - sum(lens))))
+    return lens
+
+
+def varlen_inputs(lengths, H, dk, dv, *, io="bf16", seed=5, s0_std=0.0):
+    """Packed variable-length prefill: the prefill laws over sum(lengths) tokens, laid out
+    [T_total, H, d] (beta [T_total, H]); cu_seqlens int32 [N + 1]; s0 [N, H, dk, dv] or None."""
+    Tt, N = int(sum(lengths)), len(lengths)
+    d = prefill_inputs(1, Tt, H, dk, dv, io=io, seed=seed)
+    out = {n: d[n][0] for n in ("q", "k", "v", "g", "beta")}
+    out["cu_seqlens"] = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    out["s0"] = torch.from_numpy(_normal(seed, "s0", (N, H, dk, dv), std=s0_std)) if s0_std > 0 else None
+    out["A_log"] = d["A_log"]
+    return out
+
+
+# The workloads, by what they are.
 WORKLOADS = {
     "recurrence_f32_B1_T256_H2_d64": dict(kind="prefill", io="f32", B=1, T=256, H=2, dk=64, dv=64,
                                            s0_std=0.0, seed=0),
@@ -173,4 +195,7 @@ WORKLOADS = {
                                           steps=20, s0_std=0.02, seed=3),
     "layer_bf16_B2_T16384_H96_d128": dict(kind="layer", io="bf16", B=2, T=16384, H=96, dk=128,
                                           dv=128, conv_std=0.5, seed=4),
+    # the headline prefill's 32768 tokens per step, packed as sequences of 1..4096 tokens
+    "varlen_bf16_T32768_H96_d128": dict(kind="varlen", io="bf16", total=32768, max_len=4096, H=96,
+                                        dk=128, dv=128, s0_std=0.0, seed=5),
 }

@@ -44,14 +44,16 @@ def _load():
     lib.kda_forward_chunked.argtypes = [vp] * 8 + [i] * 6 + [i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 4 + [i, vp]
+    lib.kda_forward_chunked_varlen.restype = i
+    lib.kda_forward_chunked_varlen.argtypes = [vp] * 9 + [i] * 6 + [i, vp]
     lib.kda_layer_workspace_size.restype = i
     lib.kda_layer_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
     lib.kda_layer_forward.restype = i
-    lib.kda_layer_forward.argtypes = [vp] * 12 + [f] + [vp] * 4 + [sz] + [i] * 5 + [i, vp]
+    lib.kda_layer_forward.argtypes = [vp] * 9 + [f] + [vp] * 3 + [f] + [vp] * 4 + [sz] + [i] * 5 + [i, vp]
     lib.kda_layer_forward_noalloc.restype = i
-    lib.kda_layer_forward_noalloc.argtypes = [vp] * 12 + [f] + [vp] * 3 + [i] * 5 + [i, vp]
+    lib.kda_layer_forward_noalloc.argtypes = [vp] * 9 + [f] + [vp] * 3 + [f] + [vp] * 3 + [i] * 5 + [i, vp]
     lib.kda_check_device_error.restype = i
-    lib.kda_layer_decode_step.argtypes = [vp] * 15 + [f] + [vp] * 2 + [i] * 4 + [i, vp]
+    lib.kda_layer_decode_step.argtypes = [vp] * 12 + [f] + [vp] * 3 + [f] + [vp] * 2 + [i] * 4 + [i, vp]
     lib.kda_layer_decode_step.restype = i
     lib.kda_check_device_error.argtypes = [vp]
     return lib
@@ -61,7 +63,8 @@ _lib = _load()
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_abi_version", "kda_forward_chunked",
                     "kda_decode_step", "kda_layer_workspace_size", "kda_layer_forward",
-                    "kda_layer_forward_noalloc", "kda_check_device_error")
+                    "kda_layer_forward_noalloc", "kda_layer_decode_step", "kda_forward_chunked_varlen",
+                    "kda_check_device_error")
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 
@@ -131,6 +134,35 @@ def kda_forward_chunked(q, k, v, g, beta, initial_state=None, out=None, final_st
     return out, final_state
 
 
+def kda_forward_chunked_varlen(q, k, v, g, beta, cu_seqlens, initial_state=None, out=None,
+                               final_state=None, *, chunk=64, stream=None):
+    """Chunked prefill of N packed sequences.  q, k, g: [T_total, H, dk]; v: [T_total, H, dv];
+    beta: [T_total, H] (io dtype); cu_seqlens: int32 CUDA tensor [N + 1] of sequence offsets
+    (0 .. T_total, non-decreasing); initial_state / final_state: [N, H, dk, dv] fp32 or None.
+    Returns (out [T_total, H, dv], final_state)."""
+    Tt, H, dk = q.shape
+    dv = v.shape[-1]
+    io = q.dtype
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a 1-D tensor of N + 1 >= 2 offsets")
+    N = cu_seqlens.numel() - 1
+    _need(cu_seqlens, (N + 1,), torch.int32, "cu_seqlens")
+    for t, s, n in ((q, (Tt, H, dk), "q"), (k, (Tt, H, dk), "k"), (g, (Tt, H, dk), "g"),
+                    (v, (Tt, H, dv), "v"), (beta, (Tt, H), "beta")):
+        _need(t, s, io, n)
+    _need(initial_state, (N, H, dk, dv), torch.float32, "initial_state", allow_none=True)
+    if out is None:
+        out = torch.empty((Tt, H, dv), dtype=io, device=q.device)
+    _need(out, (Tt, H, dv), io, "out")
+    _need(final_state, (N, H, dk, dv), torch.float32, "final_state", allow_none=True)
+    _check(_lib.kda_forward_chunked_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                           _ptr(initial_state), _ptr(out), _ptr(final_state),
+                                           _ptr(cu_seqlens), N, Tt, H, dk, dv, chunk, _io_code(io),
+                                           _stream(stream)),
+           "kda_forward_chunked_varlen")
+    return out, final_state
+
+
 def kda_decode_step(q, k, v, g, beta, state, out=None, *, stream=None):
     """One decode step; ``state`` [B, H, dk, dv] fp32 is updated in place.  Returns out [B, H, dv]."""
     B, H, dk = q.shape
@@ -149,6 +181,11 @@ def kda_decode_step(q, k, v, g, beta, state, out=None, *, stream=None):
     return out
 
 
+def _lb(bound):
+    """The gate's lower bound as the C ABI takes it: -inf for none."""
+    return float("-inf") if bound is None else float(bound)
+
+
 def kda_layer_workspace_size(B, T, H, dk, dv, dtype):
     n = ctypes.c_size_t(0)
     _check(_lib.kda_layer_workspace_size(B, T, H, dk, dv, _io_code(dtype), ctypes.byref(n)),
@@ -158,9 +195,10 @@ def kda_layer_workspace_size(B, T, H, dk, dv, dtype):
 
 def kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
                       o_gate_raw, o_norm_w=None, *, norm_eps=1e-6, initial_state=None, out=None,
-                      final_state=None, workspace=None, stream=None):
+                      final_state=None, workspace=None, gate_lower_bound=None, stream=None):
     """KDA layer core (prologue -> chunked gated delta rule -> epilogue).  Returns (out, final_state).
-    ``workspace`` (a uint8 CUDA tensor) is allocated with torch when not given."""
+    ``workspace`` (a uint8 CUDA tensor) is allocated with torch when not given.
+    ``gate_lower_bound`` (<= 0, e.g. -5.0) bounds every log-decay g from below; None: unbounded."""
     B, T, H, dk = g_raw.shape
     dv = o_gate_raw.shape[-1]
     io = g_raw.dtype
@@ -184,15 +222,15 @@ def kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.kda_layer_forward(
         _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
-        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
-        float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(workspace),
+        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _lb(gate_lower_bound), _ptr(b_raw), _ptr(o_gate_raw),
+        _ptr(o_norm_w), float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(workspace),
         ws_bytes, B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward")
     return out, final_state
 
 
 def kda_layer_decode_step(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cache_q, cache_k, cache_v, g_raw,
                           A_log, dt_bias, b_raw, o_gate_raw, state, o_norm_w=None, *, norm_eps=1e-6,
-                          out=None, stream=None):
+                          out=None, gate_lower_bound=None, stream=None):
     """One decode step of the layer core.  ``cache_*`` [B, 3, H*d] (io dtype, oldest tap first)
     and ``state`` [B, H, dk, dv] fp32 are updated in place.  Returns out [B, H, dv]."""
     B, H, dk = g_raw.shape
@@ -216,14 +254,14 @@ def kda_layer_decode_step(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, cache_q, 
     _check(_lib.kda_layer_decode_step(
         _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
         _ptr(cache_q), _ptr(cache_k), _ptr(cache_v), _ptr(g_raw), _ptr(A_log), _ptr(dt_bias),
-        _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w), float(norm_eps), _ptr(state), _ptr(out),
+        _lb(gate_lower_bound), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w), float(norm_eps), _ptr(state), _ptr(out),
         B, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_decode_step")
     return out
 
 
 def kda_layer_forward_noalloc(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,
                               b_raw, o_gate_raw, o_norm_w=None, *, norm_eps=1e-6, initial_state=None,
-                              out=None, final_state=None, stream=None):
+                              out=None, final_state=None, gate_lower_bound=None, stream=None):
     """kda_layer_forward with its scratch in the library's own fixed device buffer (no
     workspace argument, no allocation inside the call except ``out`` when it is not given —
     pass ``out`` to allocate nothing at all).  Sizes needing more than NOALLOC_SCRATCH_BYTES
@@ -247,8 +285,8 @@ def kda_layer_forward_noalloc(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw
     _need(out, (B, T, H, dv), io, "out")
     _check(_lib.kda_layer_forward_noalloc(
         _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
-        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _ptr(b_raw), _ptr(o_gate_raw), _ptr(o_norm_w),
-        float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state),
+        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _lb(gate_lower_bound), _ptr(b_raw), _ptr(o_gate_raw),
+        _ptr(o_norm_w), float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state),
         B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward_noalloc")
     return out, final_state
 
@@ -260,6 +298,7 @@ def kda_check_device_error(stream=None):
 
 # short names
 forward_chunked = kda_forward_chunked
+forward_chunked_varlen = kda_forward_chunked_varlen
 decode_step = kda_decode_step
 layer_forward = kda_layer_forward
 layer_workspace_size = kda_layer_workspace_size

@@ -81,6 +81,32 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
                                  int chunk, kda_dtype_t io, kda_stream_t stream);
 
 /*
+ * kda_forward_chunked_varlen — chunked prefill of N packed sequences of different lengths
+ * (the variable-length batches that segment ids or a padding mask describe; the MaxText
+ * port of the Kimi-K3 model rejects packing for KDA).  Each sequence runs the recurrence
+ * from its own initial state; no state crosses a sequence boundary.
+ *   q, k, g       [T_total, H, dk]  io dtype, the sequences' tokens back to back
+ *   v             [T_total, H, dv]  io dtype
+ *   beta          [T_total, H]      io dtype
+ *   cu_seqlens    [N + 1] int32, DEVICE memory: sequence n is tokens cu_seqlens[n] ..
+ *                 cu_seqlens[n + 1] - 1.  Expected non-decreasing from 0 to T_total.  The
+ *                 values are read on the device only and are not checked; every offset is
+ *                 clamped into [0, T_total] (and each end to at least its start), so no
+ *                 access leaves the buffers, but other malformed arrays give unspecified
+ *                 results.  A zero-length sequence passes its initial state through.
+ *   initial_state [N, H, dk, dv]  fp32 or NULL (zeros)
+ *   out           [T_total, H, dv]  io dtype (written at every token of the N sequences)
+ *   final_state   [N, H, dk, dv]  fp32 or NULL; may equal initial_state
+ *   chunk         must be 64.
+ * Supported: as kda_forward_chunked.  T_total = 0: final_state receives initial_state.
+ */
+kda_status_t kda_forward_chunked_varlen(const void *q, const void *k, const void *v, const void *g,
+                                        const void *beta, const float *initial_state, void *out,
+                                        float *final_state, const int *cu_seqlens, int N,
+                                        int T_total, int H, int dk, int dv, int chunk,
+                                        kda_dtype_t io, kda_stream_t stream);
+
+/*
  * One decode step: the recurrence for a single new token per sequence, with the
  * state updated in place (read once, written once).
  *   q, k, g [B, H, dk] io dtype; v, out [B, H, dv] io dtype; beta [B, H] io dtype;
@@ -103,7 +129,8 @@ kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_d
  *   prologue  q = l2norm(SiLU(conv_q * q_raw)), k = l2norm(SiLU(conv_k * k_raw)),
  *             v = SiLU(conv_v * v_raw)   (depthwise causal conv, kernel 4, zero history,
  *                                          PyTorch Conv1d tap order; l2norm eps 1e-6)
- *             g = -exp(A_log[h]) * softplus(g_raw + dt_bias),  beta = sigmoid(b_raw)
+ *             g = max(-exp(A_log[h]) * softplus(g_raw + dt_bias), gate_lower_bound),
+ *             beta = sigmoid(b_raw)
  *   epilogue  out = o_norm_w * cast_io(o * rsqrt(mean_dv(o^2) + norm_eps)) * sigmoid(o_gate_raw)
  * (open-model-atlas "Kimi-K3" linear_attn_config: short_conv_kernel_size 4;
  *  atlas.klimoza.dev KimiRMSNorm excerpt; maxtext PR #5543 sigmoid output gate.)
@@ -111,6 +138,10 @@ kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_d
  *   conv_q, conv_k [H*dk, 4] fp32             conv_v      [H*dv, 4]     fp32
  *   g_raw         [B, T, H, dk] io dtype      A_log       [H]           fp32
  *   dt_bias       [H*dk] fp32 or NULL (zero)  b_raw       [B, T, H]     io dtype
+ *   gate_lower_bound  a lower bound on every log-decay g, <= 0; -INFINITY for none.  (The
+ *                 Kimi-K3 linear-attention config sets gate_lower_bound = -5.0 and gives no
+ *                 formula; it is read as a bound on g itself, so that no token decays the
+ *                 state by more than exp(bound) per channel.)  NaN or > 0: KDA_ERR_INVALID_ARG.
  *   o_gate_raw    [B, T, H, dv] io dtype      o_norm_w    [dv] fp32 or NULL (ones)
  *   initial_state / final_state as in kda_forward_chunked.
  *   out           [B, T, H, dv] io dtype (written)
@@ -121,9 +152,9 @@ kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_d
 kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void *v_raw,
                                const float *conv_q, const float *conv_k, const float *conv_v,
                                const void *g_raw, const float *A_log, const float *dt_bias,
-                               const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
-                               float norm_eps, const float *initial_state, void *out,
-                               float *final_state, void *workspace, size_t workspace_bytes,
+                               float gate_lower_bound, const void *b_raw, const void *o_gate_raw,
+                               const float *o_norm_w, float norm_eps, const float *initial_state,
+                               void *out, float *final_state, void *workspace, size_t workspace_bytes,
                                int B, int T, int H, int dk, int dv, kda_dtype_t io,
                                kda_stream_t stream);
 
@@ -151,7 +182,7 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
 kda_status_t kda_layer_forward_noalloc(const void *q_raw, const void *k_raw, const void *v_raw,
                                        const float *conv_q, const float *conv_k,
                                        const float *conv_v, const void *g_raw, const float *A_log,
-                                       const float *dt_bias, const void *b_raw,
+                                       const float *dt_bias, float gate_lower_bound, const void *b_raw,
                                        const void *o_gate_raw, const float *o_norm_w,
                                        float norm_eps, const float *initial_state, void *out,
                                        float *final_state, int B, int T, int H, int dk, int dv,
@@ -173,6 +204,7 @@ kda_status_t kda_layer_forward_noalloc(const void *q_raw, const void *k_raw, con
  *   conv_q, conv_k [H*dk, 4] fp32            conv_v       [H*dv, 4] fp32
  *   g_raw         [B, H, dk] io dtype        A_log        [H] fp32
  *   dt_bias       [H*dk] fp32 or NULL        b_raw        [B, H] io dtype
+ *   gate_lower_bound  as in kda_layer_forward (-INFINITY for none)
  *   o_gate_raw    [B, H, dv] io dtype        o_norm_w     [dv] fp32 or NULL (ones)
  *   state         [B, H, dk, dv] fp32, updated in place
  *   out           [B, H, dv] io dtype (written)
@@ -183,9 +215,9 @@ kda_status_t kda_layer_forward_noalloc(const void *q_raw, const void *k_raw, con
 kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const void *v_raw,
                                    const float *conv_q, const float *conv_k, const float *conv_v,
                                    void *cache_q, void *cache_k, void *cache_v, const void *g_raw,
-                                   const float *A_log, const float *dt_bias, const void *b_raw,
-                                   const void *o_gate_raw, const float *o_norm_w, float norm_eps,
-                                   float *state, void *out, int B, int H, int dk, int dv,
+                                   const float *A_log, const float *dt_bias, float gate_lower_bound,
+                                   const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
+                                   float norm_eps, float *state, void *out, int B, int H, int dk, int dv,
                                    kda_dtype_t io, kda_stream_t stream);
 
 /*

@@ -52,7 +52,7 @@ def test_status_strings(lib):
         s = lib.kda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.kda_status_string(99) == b"unknown status"
-    assert lib.kda_abi_version() == 100
+    assert lib.kda_abi_version() == 101
 
 
 P = ctypes.c_void_p
@@ -81,6 +81,21 @@ def test_forward_chunked_rejects_bad_arguments(lib):
     assert _chunked(lib, B=1 << 20, T=1 << 20) == 2
 
 
+def test_forward_chunked_varlen_rejects_bad_arguments(lib):
+    def call(cu=A16, q=A16, N=3, Tt=100, chunk=64, dk=128, s0=None, io=1):
+        return lib.kda_forward_chunked_varlen(q, A16, A16, A16, A16, s0, A16, None, cu, N, Tt, 2, dk, 128,
+                                              chunk, io, None)
+    assert call(cu=None) == 1           # offsets are required
+    assert call(q=None) == 1
+    assert call(N=0) == 1
+    assert call(Tt=-1) == 1
+    assert call(io=5) == 1
+    assert call(chunk=16) == 2
+    assert call(dk=32) == 2
+    assert call(cu=MIS) == 3
+    assert call(s0=MIS) == 3
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A16] * 7
     ok = lambda **kw: lib.kda_decode_step(*[kw.get(n, a) for n, a in zip("qkvgbso", args)],
@@ -96,14 +111,17 @@ def test_decode_rejects_bad_arguments(lib):
 def test_layer_decode_rejects_bad_arguments(lib):
     names = ["qr", "kr", "vr", "cq", "ck", "cv", "xq", "xk", "xv", "g", "al", "dt", "b", "z", "w"]
 
-    def step(eps=1e-6, **kw):
+    def step(eps=1e-6, lb=-5.0, **kw):
         ptrs = [kw.get(n, None if n in ("dt", "w") else A16) for n in names]
+        ptrs.insert(12, ctypes.c_float(lb))
         return lib.kda_layer_decode_step(*ptrs, ctypes.c_float(eps), kw.get("S", A16), kw.get("o", A16),
                                          kw.get("B", 2), kw.get("H", 3), kw.get("dk", 128), kw.get("dv", 128),
                                          kw.get("io", 1), None)
     assert step(S=None) == 1
     assert step(xk=None) == 1
     assert step(eps=-1.0) == 1
+    assert step(lb=0.5) == 1            # a bound above 0 would let the state grow
+    assert step(lb=float("nan")) == 1
     assert step(H=0) == 1
     assert step(dk=64, dv=64) == 2      # d = 128 only
     assert step(xv=MIS) == 3
@@ -119,12 +137,15 @@ def test_layer_workspace_and_argument_checks(lib):
     assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, None) == 1
     assert lib.kda_layer_workspace_size(2, 16, 3, 100, 128, 1, ctypes.byref(n)) == 2
 
-    def layer(ws=A16, ws_bytes=1 << 40, q=A16, eps=1e-6, **kw):
-        return lib.kda_layer_forward(q, A16, A16, A16, A16, A16, A16, A16, None, A16, A16, None,
+    def layer(ws=A16, ws_bytes=1 << 40, q=A16, eps=1e-6, lb=float("-inf"), **kw):
+        return lib.kda_layer_forward(q, A16, A16, A16, A16, A16, A16, A16, None, ctypes.c_float(lb),
+                                     A16, A16, None,
                                      ctypes.c_float(eps), None, A16, None, ws, ws_bytes,
                                      kw.get("B", 1), kw.get("T", 16), kw.get("H", 2), 128, 128, 1, None)
     assert layer(q=None) == 1
     assert layer(eps=-1.0) == 1
+    assert layer(lb=1.0) == 1
+    assert layer(lb=float("nan")) == 1
     assert layer(q=MIS) == 3
     assert layer(ws=None) == 6
     assert layer(ws_bytes=16) == 6

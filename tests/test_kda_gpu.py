@@ -297,10 +297,81 @@ def test_decode_chain_equals_prefill(kda):
     torch.testing.assert_close(S, s_p, rtol=1e-4, atol=1e-5)
 
 
+# ------------------------------------------------------------------------ packed variable length
+
+
+def run_varlen(kda, d, with_final=True):
+    dev = "cuda"
+    q, k, v, g, beta = (d[n].to(dev) for n in ("q", "k", "v", "g", "beta"))
+    cu = d["cu_seqlens"].to(dev)
+    s0 = None if d["s0"] is None else d["s0"].to(dev)
+    N, H, dk, dv = cu.numel() - 1, q.shape[1], q.shape[2], v.shape[2]
+    sT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if with_final else None
+    out, sT = kda.kda_forward_chunked_varlen(q, k, v, g, beta, cu, s0, None, sT)
+    kda.kda_check_device_error()
+    return out, sT
+
+
+def oracle_varlen(d):
+    return oracle.recurrent_varlen(f64(d["q"]), f64(d["k"]), f64(d["v"]), f64(d["g"]), f64(d["beta"]),
+                                   d["cu_seqlens"].numpy(), None if d["s0"] is None else f64(d["s0"]))
+
+
+# lengths: empty first and middle sequences, 1 token, one short of / exactly / one past a
+# chunk, several chunks with a ragged tail, and a ragged last sequence
+VARLEN_LENS = [0, 1, 63, 64, 65, 0, 130, 7, 200]
+
+
+@pytest.mark.parametrize("io,d_", [(torch.bfloat16, 128), (torch.float32, 128),
+                                   (torch.bfloat16, 64), (torch.float32, 64)])
+def test_varlen_ragged_lengths(kda, io, d_):
+    """Every token's output and every sequence's final state against the oracle run per
+    sequence (tcgen05 kernel for bf16 d = 128, exact fp32 kernels otherwise)."""
+    d = inputs.varlen_inputs(VARLEN_LENS, 3, d_, d_, io="f32" if io == torch.float32 else "bf16",
+                             seed=80 + d_, s0_std=0.05)
+    out, sT = run_varlen(kda, d)
+    ro, rs = oracle_varlen(d)
+    assert err(f64(out), ro, io) <= tol(io)
+    assert serr(f64(sT), rs, io) <= 1.0
+    # zero-length sequences pass the initial state through exactly
+    for n in (0, 5):
+        assert torch.equal(sT[n].cpu(), d["s0"][n])
+
+
+@pytest.mark.parametrize("io,d_", [(torch.bfloat16, 128), (torch.float32, 128), (torch.bfloat16, 64)])
+def test_varlen_equal_lengths_equal_the_fixed_length_call(kda, io, d_):
+    """Three packed sequences of 150 tokens give the batched B = 3, T = 150 call's results bit
+    for bit (same kernel; the packed tail chunk's foreign rows are masked)."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.varlen_inputs([150, 150, 150], 2, d_, d_, io=ioname, seed=90, s0_std=0.05)
+    ov, sv = run_varlen(kda, d)
+    fixed = {n: d[n].reshape((3, 150) + tuple(d[n].shape[1:])) for n in ("q", "k", "v", "g", "beta")}
+    fixed["s0"] = d["s0"]
+    of, sf = run_prefill(kda, fixed)
+    assert torch.equal(ov.reshape(of.shape), of)
+    assert torch.equal(sv, sf)
+
+
+def test_varlen_workload_T32768_H96_sampled(kda):
+    """The packed workload (32768 tokens of 15 sequences, 1..4096 tokens each, H = 96) in the
+    benchmark's launch shape; sampled (sequence, head) pairs against the oracle."""
+    w = inputs.WORKLOADS["varlen_bf16_T32768_H96_d128"]
+    lens = inputs.packed_lengths(w["total"], w["max_len"], w["seed"])
+    d = inputs.varlen_inputs(lens, w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    out, sT = run_varlen(kda, d)
+    cu = d["cu_seqlens"].numpy()
+    longest = int(np.argmax(lens))
+    for n, h in [(0, 0), (longest, 95), (len(lens) - 1, 17), (len(lens) // 2, 50)]:
+        a, b = int(cu[n]), int(cu[n + 1])
+        ro, rs = oracle.recurrent(*(f64(d[x][a:b, h:h + 1])[None] for x in ("q", "k", "v", "g", "beta")))
+        assert err(f64(out[a:b, h:h + 1])[None], ro, torch.bfloat16) <= 1.0
+        assert serr(f64(sT[n, h])[None, None], rs, torch.bfloat16) <= 1.0
+
+
 # ------------------------------------------------------------------------ layer
 
 
-def run_layer(kda, d, with_final=True):
+def run_layer(kda, d, with_final=True, lb=None):
     dev = "cuda"
     to = lambda x: None if x is None else x.to(dev)
     B, T, H, dk = d["g_raw"].shape
@@ -309,18 +380,19 @@ def run_layer(kda, d, with_final=True):
     out, sT = kda.kda_layer_forward(
         to(d["q_raw"]), to(d["k_raw"]), to(d["v_raw"]), to(d["conv_q"]), to(d["conv_k"]),
         to(d["conv_v"]), to(d["g_raw"]), to(d["A_log"]), to(d["dt_bias"]), to(d["b_raw"]),
-        to(d["o_gate_raw"]), to(d["o_norm_w"]), initial_state=to(d["s0"]), final_state=sT)
+        to(d["o_gate_raw"]), to(d["o_norm_w"]), initial_state=to(d["s0"]), final_state=sT,
+        gate_lower_bound=lb)
     kda.kda_check_device_error()
     return out, sT
 
 
-def oracle_layer(d, io, heads=None):
+def oracle_layer(d, io, heads=None, lb=None):
     a = {n: (None if d[n] is None else f64(d[n])) for n in d}
     io_bf16 = io == torch.bfloat16
     if heads is None:
         return oracle.layer(a["q_raw"], a["k_raw"], a["v_raw"], a["conv_q"], a["conv_k"], a["conv_v"],
                             a["g_raw"], a["A_log"], a["dt_bias"], a["b_raw"], a["o_gate_raw"],
-                            a["o_norm_w"], io_bf16=io_bf16, s0=a["s0"])
+                            a["o_norm_w"], io_bf16=io_bf16, s0=a["s0"], gate_lower_bound=lb)
     B, T, H, dk = a["g_raw"].shape
     dv = a["o_gate_raw"].shape[-1]
     outs, states = [], []
@@ -332,7 +404,7 @@ def oracle_layer(d, io, heads=None):
                             a["conv_v"][cv], a["g_raw"][b:b + 1, :, h:h + 1], a["A_log"][h:h + 1],
                             None if a["dt_bias"] is None else a["dt_bias"][ck], a["b_raw"][b:b + 1, :, h:h + 1],
                             a["o_gate_raw"][b:b + 1, :, h:h + 1], a["o_norm_w"], io_bf16=io_bf16,
-                            s0=None if a["s0"] is None else a["s0"][b:b + 1, h:h + 1])
+                            s0=None if a["s0"] is None else a["s0"][b:b + 1, h:h + 1], gate_lower_bound=lb)
         outs.append(o[0, :, 0])
         states.append(s[0, 0])
     return np.stack(outs, 1)[None], np.stack(states, 0)[None]
@@ -349,6 +421,28 @@ def test_layer_small(kda, io, d_, T):
     ro, rs = oracle_layer(d, io)
     assert err(f64(out), ro, io, stored_bf16=2) <= tol(io)
     assert serr(f64(sT), rs, io) <= 1.0
+
+
+def clamped_fraction(d, lb):
+    g = oracle.gate(f64(d["g_raw"]), f64(d["A_log"]), None if d["dt_bias"] is None else f64(d["dt_bias"]))
+    return float(np.mean(g < lb))
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d_", [64, 128])
+def test_layer_gate_lower_bound(kda, io, d_):
+    """gate_lower_bound = -5 (the Kimi-K3 linear-attention config's value) on a draw where a
+    good part of the log-decays fall below it: the layer equals the oracle with the bound."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.layer_inputs(2, 150, 3, d_, d_, io=ioname, seed=70 + d_, s0_std=0.05,
+                            dt_bias_std=0.5, gain_std=0.2)
+    assert clamped_fraction(d, -5.0) > 0.05
+    out, sT = run_layer(kda, d, lb=-5.0)
+    ro, rs = oracle_layer(d, io, lb=-5.0)
+    assert err(f64(out), ro, io, stored_bf16=2) <= tol(io)
+    assert serr(f64(sT), rs, io) <= 1.0
+    ru, _ = oracle_layer(d, io)
+    assert np.max(np.abs(ru - ro)) > 10 * np.max(np.abs(f64(out) - ro))   # the bound matters
 
 
 def test_layer_workload_B2_T16384_H96_sampled_heads(kda):
@@ -376,8 +470,9 @@ def test_layer_zero_gate_input_halves_output(kda):
 # ------------------------------------------------------------------------ layer decode (conv cache)
 
 
+@pytest.mark.parametrize("lb", [None, -2.0])
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
-def test_layer_decode_steps_equal_layer_over_the_same_tokens(kda, io):
+def test_layer_decode_steps_equal_layer_over_the_same_tokens(kda, io, lb):
     """n layer-decode steps from an empty conv cache give the layer's outputs over those n
     tokens and its final state; the cache ends holding the last three raw tokens, bit for bit."""
     ioname = "f32" if io == torch.float32 else "bf16"
@@ -392,11 +487,13 @@ def test_layer_decode_steps_equal_layer_over_the_same_tokens(kda, io):
         o = kda.kda_layer_decode_step(
             to(L["q_raw"][:, t]), to(L["k_raw"][:, t]), to(L["v_raw"][:, t]), to(L["conv_q"]), to(L["conv_k"]),
             to(L["conv_v"]), *caches, to(L["g_raw"][:, t]), to(L["A_log"]), to(L["dt_bias"]), to(L["b_raw"][:, t]),
-            to(L["o_gate_raw"][:, t]), state, to(L["o_norm_w"]))
+            to(L["o_gate_raw"][:, t]), state, to(L["o_norm_w"]), gate_lower_bound=lb)
         outs.append(o)
     kda.kda_check_device_error()
     out = torch.stack(outs, 1)
-    ro, rs = oracle_layer(L, io)
+    if lb is not None:
+        assert clamped_fraction(L, lb) > 0.05
+    ro, rs = oracle_layer(L, io, lb=lb)
     assert err(f64(out), ro, io, stored_bf16=2) <= 1.0
     assert serr(f64(state), rs, io) <= 1.0
     for c, n in zip(caches, ("q_raw", "k_raw", "v_raw")):
