@@ -51,6 +51,7 @@ def _load():
             d = ctypes.c_double
             sz = ctypes.c_size_t
             lib.kda_oracle_recurrent.argtypes = [_dp] * 8 + [i] * 7
+            lib.kda_oracle_recurrent_backward.argtypes = [_dp] * 14 + [i] * 6
             lib.kda_oracle_decode.argtypes = [_dp] * 7 + [i] * 5
             lib.kda_oracle_short_conv_silu.argtypes = [_dp] * 3 + [i] * 5
             lib.kda_oracle_l2norm.argtypes = [_dp, _dp, sz, i, d]
@@ -99,6 +100,27 @@ def recurrent(q, k, v, g, beta, s0=None, *, delta=True, nthreads=0):
         B, T, H, dk, dv, 1 if delta else 0, nthreads,
     )
     return o, sT
+
+
+def recurrent_backward(q, k, v, g, beta, s0, d_o, d_sT=None, *, nthreads=0):
+    """Gradients of the recurrence by reverse mode, token by token, in fp64.
+
+    Arguments as ``recurrent`` plus d_o = dL/do [B, T, H, dv] and d_sT = dL/dS_T
+    [B, H, dk, dv] (None: zero).  Returns dict dq, dk, dv, dg, dbeta, ds0.
+    """
+    q, k, v, g, beta, s0, d_o, d_sT = map(_f64, (q, k, v, g, beta, s0, d_o, d_sT))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert d_o.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    assert d_sT is None or d_sT.shape == (B, H, dk, dv)
+    out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v), "dg": np.zeros_like(g),
+           "dbeta": np.zeros_like(beta), "ds0": np.zeros((B, H, dk, dv))}
+    _load().kda_oracle_recurrent_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(s0), _ptr(d_o), _ptr(d_sT),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]),
+        _ptr(out["ds0"]), B, T, H, dk, dv, nthreads,
+    )
+    return out
 
 
 def recurrent_varlen(q, k, v, g, beta, cu_seqlens, s0=None, *, nthreads=0):

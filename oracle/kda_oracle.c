@@ -147,6 +147,116 @@ void kda_oracle_recurrent(const double *q, const double *k, const double *v, con
     }
 }
 
+/* Gradients of the recurrence (reverse mode, token by token, exact in fp64).
+ * Given dO = dL/do [B, T, H, dv] and dST = dL/dS_T [B, H, dk, dv] (NULL: zero), writes
+ * dq, dk, dg [B, T, H, dk], dv [B, T, H, dv], dbeta [B, T, H] and ds0 = dL/dS_0
+ * [B, H, dk, dv] (NULL: not wanted).  The pages' training runs differentiate the layer
+ * (maxtext PR #5550, its jax.grad test and the C4 training steps); the steps below are
+ * the chain rule applied to each line of the forward step, last token first:
+ *   S' = Diag(a) S_{t-1}, a = exp(g_t);  r = S'^T k;  u = beta (v - r);  S_t = S' + k u^T;
+ *   o_t = S_t^T q.
+ * The forward states S_0 .. S_{T-1} are kept (one head at a time). */
+void kda_oracle_recurrent_backward(const double *q, const double *k, const double *v,
+                                   const double *g, const double *beta, const double *s0,
+                                   const double *dO, const double *dST, double *dq, double *dk,
+                                   double *dv_, double *dg, double *dbeta, double *ds0, int B,
+                                   int T, int H, int dk_, int dv, int nthreads)
+{
+    set_threads(nthreads);
+    const size_t sk = (size_t)H * dk_, sv = (size_t)H * dv, DD = (size_t)dk_ * dv;
+#pragma omp parallel
+    {
+        double *Sall = (double *)malloc(sizeof(double) * DD * (size_t)(T + 1));
+        double *U = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * dv);
+        double *R = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * dv);
+        double *Sp = (double *)malloc(sizeof(double) * DD);
+        double *dS = (double *)malloc(sizeof(double) * DD);
+        double *du = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *da = (double *)malloc(sizeof(double) * (size_t)dv);
+#pragma omp for schedule(dynamic, 1)
+        for (int bh = 0; bh < B * H; ++bh) {
+            const int b = bh / H, h = bh % H;
+            const size_t tok0 = (size_t)b * T * H + h;
+            /* forward: S_0 .. S_T, u_t and r_t = S'^T k */
+            if (s0) memcpy(Sall, s0 + (size_t)bh * DD, sizeof(double) * DD);
+            else memset(Sall, 0, sizeof(double) * DD);
+            for (int t = 0; t < T; ++t) {
+                const size_t tk = (tok0 + (size_t)t * H) * dk_, tv = (tok0 + (size_t)t * H) * dv;
+                const double *Sprev = Sall + (size_t)t * DD;
+                double *Snext = Sall + (size_t)(t + 1) * DD;
+                for (int c = 0; c < dk_; ++c) {
+                    const double a = exp(g[tk + c]);
+                    for (int j = 0; j < dv; ++j) Snext[(size_t)c * dv + j] = a * Sprev[(size_t)c * dv + j];
+                }
+                const double bt = beta[tok0 + (size_t)t * H];
+                for (int j = 0; j < dv; ++j) {
+                    double r = 0.0;
+                    for (int c = 0; c < dk_; ++c) r += Snext[(size_t)c * dv + j] * k[tk + c];
+                    R[(size_t)t * dv + j] = r;
+                    U[(size_t)t * dv + j] = bt * (v[tv + j] - r);
+                }
+                for (int c = 0; c < dk_; ++c)
+                    for (int j = 0; j < dv; ++j) Snext[(size_t)c * dv + j] += k[tk + c] * U[(size_t)t * dv + j];
+            }
+            /* reverse sweep */
+            if (dST) memcpy(dS, dST + (size_t)bh * DD, sizeof(double) * DD);
+            else memset(dS, 0, sizeof(double) * DD);
+            for (int t = T - 1; t >= 0; --t) {
+                const size_t tk = (tok0 + (size_t)t * H) * dk_, tv = (tok0 + (size_t)t * H) * dv;
+                const size_t tb = tok0 + (size_t)t * H;
+                const double *St = Sall + (size_t)(t + 1) * DD, *Sprev = Sall + (size_t)t * DD;
+                const double bt = beta[tb];
+                /* o_t = S_t^T q_t:  dS_t += q do^T,  dq = S_t do */
+                for (int c = 0; c < dk_; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        dS[(size_t)c * dv + j] += q[tk + c] * dO[tv + j];
+                        acc += St[(size_t)c * dv + j] * dO[tv + j];
+                    }
+                    dq[tk + c] = acc;
+                }
+                /* S_t = S' + k u^T:  du = dS^T k,  dk = dS u */
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk_; ++c) acc += dS[(size_t)c * dv + j] * k[tk + c];
+                    du[j] = acc;
+                }
+                double dbt = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    /* u = beta (v - r) */
+                    dbt += du[j] * (v[tv + j] - R[(size_t)t * dv + j]);
+                    dv_[tv + j] = bt * du[j];
+                    da[j] = -bt * du[j];
+                }
+                dbeta[tb] = dbt;
+                for (int c = 0; c < dk_; ++c) {
+                    const double a = exp(g[tk + c]);
+                    double acc_k = 0.0, acc_g = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        const double sp = a * Sprev[(size_t)c * dv + j];
+                        acc_k += dS[(size_t)c * dv + j] * U[(size_t)t * dv + j] + sp * da[j];
+                        /* r = S'^T k:  dS' = dS + k da^T */
+                        const double dsp = dS[(size_t)c * dv + j] + k[tk + c] * da[j];
+                        /* S' = Diag(exp g) S_{t-1}:  dg_c = sum_j dS'_cj S'_cj,  dS_{t-1} = Diag(exp g) dS' */
+                        acc_g += dsp * sp;
+                        dS[(size_t)c * dv + j] = a * dsp;
+                    }
+                    dk[tk + c] = acc_k;
+                    dg[tk + c] = acc_g;
+                }
+            }
+            if (ds0) memcpy(ds0 + (size_t)bh * DD, dS, sizeof(double) * DD);
+        }
+        free(Sall);
+        free(U);
+        free(R);
+        free(Sp);
+        free(dS);
+        free(du);
+        free(da);
+    }
+}
+
 /* One decode step: the recurrence for a single token per sequence, state updated
  * in place.  q, k, g: [B, H, dk]; v, o: [B, H, dv]; beta: [B, H]; state [B, H, dk, dv]. */
 void kda_oracle_decode(const double *q, const double *k, const double *v, const double *g,

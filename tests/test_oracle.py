@@ -263,6 +263,80 @@ def test_varlen_sequences_are_isolated():
     assert np.max(np.abs(o1[6:13] - o2[6:13])) > 1e-3
 
 
+# --------------------------------------------------------------- gradients
+
+
+def _loss(q, k, v, g, beta, s0, Wo, Ws):
+    o, sT = oracle.recurrent(q, k, v, g, beta, s0)
+    return float(np.sum(Wo * o) + np.sum(Ws * sT))
+
+
+def test_backward_equals_central_differences():
+    """Every gradient of L = <Wo, o> + <Ws, S_T> against central differences of the forward
+    oracle (step 1e-6; the difference error is O(1e-12) here)."""
+    rng = np.random.default_rng(31)
+    B, T, H, dk, dv = 1, 6, 2, 4, 3
+    q, k, v, g, beta, s0 = _rand_inputs(rng, B, T, H, dk, dv, s0_std=0.5)
+    Wo = rng.standard_normal((B, T, H, dv))
+    Ws = rng.standard_normal((B, H, dk, dv))
+    gr = oracle.recurrent_backward(q, k, v, g, beta, s0, Wo, Ws)
+    args = {"q": q, "k": k, "v": v, "g": g, "beta": beta, "s0": s0}
+    eps = 1e-6
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"), ("s0", "ds0")):
+        x = args[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + eps
+            lp = _loss(**args, Wo=Wo, Ws=Ws)
+            x[idx] = old - eps
+            lm = _loss(**args, Wo=Wo, Ws=Ws)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert _rel(gr[key], fd) < 1e-7, name
+
+
+def test_backward_equals_torch_autograd():
+    """The same gradients from torch autograd through a plain fp64 token loop of the
+    recurrence (an independent route: library reverse mode, no hand-written chain rule)."""
+    rng = np.random.default_rng(32)
+    B, T, H, dk, dv = 2, 9, 2, 5, 4
+    q, k, v, g, beta, s0 = _rand_inputs(rng, B, T, H, dk, dv, s0_std=0.3)
+    Wo = rng.standard_normal((B, T, H, dv))
+    Ws = rng.standard_normal((B, H, dk, dv))
+    ts = {n: torch.tensor(x, requires_grad=True) for n, x in
+          (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("s0", s0))}
+    S = ts["s0"]
+    outs = []
+    for t in range(T):
+        Sp = torch.exp(ts["g"][:, t])[..., None] * S
+        r = torch.einsum("bhcj,bhc->bhj", Sp, ts["k"][:, t])
+        u = ts["beta"][:, t][..., None] * (ts["v"][:, t] - r)
+        S = Sp + ts["k"][:, t][..., None] * u[:, :, None, :]
+        outs.append(torch.einsum("bhcj,bhc->bhj", S, ts["q"][:, t]))
+    o = torch.stack(outs, 1)
+    (torch.sum(torch.tensor(Wo) * o) + torch.sum(torch.tensor(Ws) * S)).backward()
+    gr = oracle.recurrent_backward(q, k, v, g, beta, s0, Wo, Ws)
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("g", "dg"), ("beta", "dbeta"), ("s0", "ds0")):
+        assert _rel(gr[key], ts[name].grad.numpy()) < 1e-12, name
+
+
+def test_backward_without_decay_or_write_is_a_readout():
+    """g = 0, beta = 0: o_t = S_0^T q_t, so dq_t = S_0 do_t, dS_0 = dS_T + sum_t q_t do_t^T,
+    and nothing flows to v or k (u = 0 and the correction is scaled by beta = 0)."""
+    rng = np.random.default_rng(33)
+    B, T, H, dk, dv = 1, 5, 1, 4, 3
+    q, k, v, _, _, s0 = _rand_inputs(rng, B, T, H, dk, dv, s0_std=1.0)
+    g = np.zeros((B, T, H, dk))
+    beta = np.zeros((B, T, H))
+    Wo = rng.standard_normal((B, T, H, dv))
+    Ws = rng.standard_normal((B, H, dk, dv))
+    gr = oracle.recurrent_backward(q, k, v, g, beta, s0, Wo, Ws)
+    assert _rel(gr["dq"], np.einsum("bhcj,bthj->bthc", s0, Wo)) < 1e-14
+    assert _rel(gr["ds0"], Ws + np.einsum("bthc,bthj->bhcj", q, Wo)) < 1e-14
+    assert np.all(gr["dv"] == 0.0) and np.all(gr["dk"] == 0.0)
+
+
 def test_state_norm_bound():
     """||k|| = 1, beta in [0, 1], g <= 0  =>  ||S_t||_2 <= ||S_{t-1}||_2 + beta_t ||v_t||."""
     rng = np.random.default_rng(13)
