@@ -50,6 +50,10 @@ L2_BYTES = 126 * 1024 * 1024
 #   chunked FLOPs as issued on full 64-row tiles: 10*C*d + 6*d^2 = 180224 per token-head.
 PREFILL_BYTES_PER_TOKEN_HEAD = 1282
 LAYER_BYTES_PER_TOKEN_HEAD = 1538
+# backward, per token-head at d = 128 (16-token chunks): the state products issued by the
+# forward sweep and the reverse sweep (9 d^2 multiply-adds) and the chunk-local ones
+# (12 * 16 * d), counted as 2 FLOP per multiply-add
+BWD_FLOPS_PER_TOKEN_HEAD = 2 * (9 * 128 * 128 + 12 * 16 * 128)
 FLOPS_PER_TOKEN_HEAD = 180224
 
 
@@ -60,7 +64,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--skip", default="", help="comma list of: varlen,decode,layer_decode,layer,e2e,cpu")
+    ap.add_argument("--skip", default="", help="comma list of: varlen,backward,decode,layer_decode,layer,e2e,cpu")
     return ap.parse_args()
 
 
@@ -318,6 +322,45 @@ def run_ours(args):
         del xv, ov, sv, dl
         torch.cuda.empty_cache()
 
+    # ------------------------------------------------------------------ backward (gradients)
+    if "backward" not in skip:
+        wb = inputs.WORKLOADS[PREFILL]
+        Bb, Tb, Hb, db_ = wb["B"], wb["T"], wb["H"], wb["dk"]
+        dbk = inputs.prefill_inputs(Bb, Tb, Hb, db_, db_, io=wb["io"], seed=wb["seed"])
+        xb = {n: dbk[n].to(dev) for n in ("q", "k", "v", "g", "beta")}
+        gen = torch.Generator().manual_seed(7)
+        dO_b = torch.randn((Bb, Tb, Hb, db_), generator=gen).to(torch.bfloat16).to(dev)
+        grads = {n: torch.empty_like(xb[m]) for n, m in (("dq", "q"), ("dk", "k"), ("dv", "v"), ("dg", "g"),
+                                                          ("dbeta", "beta"))}
+        ds0 = torch.empty((Bb, Hb, db_, db_), dtype=torch.float32, device=dev)
+        ws_b = torch.empty(kda.kda_backward_workspace_size(Bb, Tb, Hb, db_, db_, torch.bfloat16),
+                           dtype=torch.uint8, device=dev)
+
+        def backward_step():
+            kda.kda_backward_chunked(xb["q"], xb["k"], xb["v"], xb["g"], xb["beta"], dO_b, None, None,
+                                     grads=grads, d_initial_state=ds0, workspace=ws_b, stream=stream)
+
+        nb = max(1, args.steps // 4)
+        total_b, per_b = timed(torch, backward_step, nb, max(1, args.warmup // 3), stream, barrier)
+        kda.kda_check_device_error(stream)
+        ms_b = max_over_ranks(total_b / nb)
+        lms_b = max_over_ranks(statistics.mean(per_b))
+        flops_b = Bb * Tb * Hb * BWD_FLOPS_PER_TOKEN_HEAD
+        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        ach_b = flops_b / (lms_b / 1e3) / 1e12
+        res["backward"] = {
+            "workload": "kda_backward_chunked B=4 T=8192 H=96 dk=dv=128 bf16 (the prefill workload, "
+                        "dO ~ N(0,1) bf16, zero initial state), fp32 arithmetic on CUDA cores",
+            "value": round(aggregate_rate(Bb * Tb, ms_b, ws), 1), "unit": "tokens/s", "ms_per_step": round(ms_b, 3),
+            "roofline": {"bound": "alu", "achieved": round(ach_b, 2), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(ach_b / alu_peak, 4), "traffic": traffic_for("kda_backward"),
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                         "kernel": "kda_backward", "launch_ms": round(lms_b, 3), "flops_per_launch": flops_b,
+                         "workspace_bytes": ws_b.numel()}}
+        launches_per["backward"] = nb
+        del xb, dO_b, grads, ds0, ws_b, dbk
+        torch.cuda.empty_cache()
+
     # ------------------------------------------------------------------ decode
     if "decode" not in skip:
         wd = inputs.WORKLOADS[DECODE]
@@ -437,7 +480,8 @@ def run_ours(args):
         cpu = cpu_baseline_prefill()
 
     gpu_launches = args.steps * (launches_per["prefill"] + launches_per.get("varlen", 0)) + \
-        launches_per.get("decode", 0) + launches_per.get("layer_decode", 0) + launches_per.get("layer", 0)
+        launches_per.get("backward", 0) + launches_per.get("decode", 0) + launches_per.get("layer_decode", 0) + \
+        launches_per.get("layer", 0)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),

@@ -116,6 +116,44 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
     return cuda_status(kda::launch_chunk_simt(a, s));
 }
 
+kda_status_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
+                                         size_t *bytes)
+{
+    if (!bytes) return KDA_ERR_INVALID_ARG;
+    kda_status_t st = check_dims(B, T, H, dk, dv, io);
+    if (st != KDA_OK) return st;
+    if (dk != dv) return KDA_ERR_UNSUPPORTED;
+    *bytes = kda::backward_workspace_bytes(B, T, H, dk);
+    return KDA_OK;
+}
+
+kda_status_t kda_backward_chunked(const void *q, const void *k, const void *v, const void *g,
+                                  const void *beta, const float *initial_state, const void *d_out,
+                                  const float *d_final_state, void *dq, void *dk_, void *dv_, void *dg,
+                                  void *dbeta, float *d_initial_state, void *workspace,
+                                  size_t workspace_bytes, int B, int T, int H, int dk, int dv,
+                                  kda_dtype_t io, kda_stream_t stream)
+{
+    kda_status_t st = check_dims(B, T, H, dk, dv, io);
+    if (st != KDA_OK) return st;
+    if (dk != dv) return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !d_out || !dq || !dk_ || !dv_ || !dg || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, initial_state, d_out, d_final_state, dq, dk_, dv_, dg, dbeta,
+                          d_initial_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) return cuda_status(kda::launch_fill_state(d_final_state, d_initial_state,
+                                                          (size_t)B * H * dk * dv, s));
+    const size_t need = kda::backward_workspace_bytes(B, T, H, dk);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255u) != 0) return KDA_ERR_MISALIGNED;
+    kda::BackwardArgs a{q, k, v, g, beta, initial_state, d_out, d_final_state, dq, dk_, dv_, dg, dbeta,
+                        d_initial_state, (float *)workspace, B, T, H, dk, io_of(io)};
+    return cuda_status(kda::launch_backward(a, s));
+}
+
 kda_status_t kda_forward_chunked_varlen(const void *q, const void *k, const void *v, const void *g,
                                         const void *beta, const float *initial_state, void *out,
                                         float *final_state, const int *cu_seqlens, int N,

@@ -1,0 +1,479 @@
+// backward.cu — gradients of the gated delta rule, chunkwise, exact fp32 on CUDA cores.
+//
+// The forward step per token t (per head):
+//   S' = Diag(exp g_t) S;   u_t = beta_t (v_t - S'^T k_t);   S_t = S' + k_t u_t^T;   o_t = S_t^T q_t
+// (the recurrence of the Kimi-K3 KDA layers; the pages' training runs differentiate it:
+//  maxtext PR #5550, its jax.grad test and the C4 training steps).
+//
+// Chunk form over BC = 16 tokens (G = in-chunk inclusive cumsum of g, G_C its last row,
+// E_ijc = exp(G_ic - G_jc) for j <= i, never above 1):
+//   Abar_ij = sum_c k_ic k_jc E_ijc (j < i)      P_ij = sum_c q_ic k_jc E_ijc (j <= i)
+//   M = (I + Diag(beta) Abar)^-1,  X = V - K^ S,  Z = Diag(beta) X,  U = M Z
+//   O = Q^ S + P U,   S_next = Diag(exp G_C) S + K~^T U
+//   with Q^ = q exp(G), K^ = k exp(G), K~ = k exp(G_C - G).
+// Reverse mode through those lines, given dO and dS_next:
+//   dU = P^T dO + K~ dS_next          dZ = M^T dU        dX = Diag(beta) dZ     dV = dX
+//   dP = tril(dO U^T)                 dA = -stril(dZ U^T)   (since M^T dM M^T = dZ U^T)
+//   dbeta = rowsum(dZ . X) + rowsum(dA . Abar),   dAbar = Diag(beta) dA
+//   dq = exp(G) (dO S^T) + sum_j dP_ij k_j E_ij
+//   dk = -exp(G) (dX S^T) + sum_j dAbar_ij k_j E_ij              ("+" part: G enters with +)
+//      + exp(G_C - G) (U dS_next^T) + sum_m (dP_mi q_m + dAbar_mi k_m) E_mi   ("-" part)
+//   dG = q dq + k dk+ - k dk-,  dG_C += sum_i k_i dk~_i + exp(G_C) rowsum(dS_next . S)
+//   dg = reverse cumsum of dG;   dS = Diag(exp G_C) dS_next + Q^^T dO - K^^T dX.
+// Every exponent is a sum of non-positive log-decays, so nothing overflows for any gate.
+//
+// One CTA of 512 threads per (b, h).  A forward sweep writes the chunk-start states to the
+// workspace (checkpoints); the reverse sweep reloads each one, recomputes the chunk's
+// forward quantities and applies the lines above, with dS held in shared memory.
+#include "common.cuh"
+#include "internal.h"
+
+namespace kda {
+namespace {
+
+constexpr int BC = 16;     // tokens per chunk
+constexpr int BNT = 512;   // threads per CTA
+
+template <int D>
+struct BwdLayout {
+    static constexpr int LD = D + 4;              // row stride of states and tiles (floats)
+    static constexpr int ST = D * LD;             // one [D][LD] state
+    static constexpr int TL = BC * LD;            // one [BC][LD] tile
+    static constexpr int CL = BC + 1;             // row stride of the BC x BC matrices
+    static constexpr int CC = BC * CL;
+    static constexpr int NB = BNT / D;            // row blocks (or value blocks) of threads
+    static constexpr int S_ = 0, DS = ST, Q = 2 * ST, K = Q + TL, G = K + TL, V = G + TL, DO = V + TL,
+                         U = DO + TL, DU = U + TL, QH = DU + TL, KH = QH + TL, KT = KH + TL;
+    static constexpr int AB = KT + TL, P = AB + CC, M = P + CC, DP = M + CC, DA = DP + CC;
+    static constexpr int BETA = DA + CC, DBETA = BETA + BC, GC = DBETA + BC, REDK = GC + D, REDS = REDK + NB * D;
+    static constexpr int FLOATS = REDS + NB * D;
+    static constexpr size_t BYTES = sizeof(float) * FLOATS;
+};
+
+struct BwdArgs {
+    const void *q, *k, *v, *g, *beta;   // io dtype
+    const float *s0;                    // [B, H, D, D] or null
+    const void *dO;                     // io dtype
+    const float *dST;                   // [B, H, D, D] or null
+    void *dq, *dk, *dv, *dg, *dbeta;    // io dtype
+    float *ds0;                         // [B, H, D, D] or null
+    float *ckpt;                        // [B, H, nchunks, D, D]
+    int T, H;
+};
+
+template <typename IO, int D>
+__global__ void __launch_bounds__(BNT, 1)
+kda_backward_kernel(BwdArgs a)
+{
+    using L = BwdLayout<D>;
+    constexpr int LD = L::LD, NB = L::NB, RPT = BC / NB, JPT = D / NB, CL = L::CL;
+    extern __shared__ __align__(16) float bsm[];
+    float *Ss = bsm + L::S_, *dSs = bsm + L::DS, *Qs = bsm + L::Q, *Ks = bsm + L::K, *Gs = bsm + L::G;
+    float *Vs = bsm + L::V, *dOs = bsm + L::DO, *Us = bsm + L::U, *dUs = bsm + L::DU;
+    float *QHs = bsm + L::QH, *KHs = bsm + L::KH, *KTs = bsm + L::KT;
+    float *ABs = bsm + L::AB, *Ps = bsm + L::P, *Ms = bsm + L::M, *dPs = bsm + L::DP, *dAs = bsm + L::DA;
+    float *BETA = bsm + L::BETA, *DBETA = bsm + L::DBETA, *GCs = bsm + L::GC;
+    float *REDK = bsm + L::REDK, *REDS = bsm + L::REDS;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int T = a.T, H = a.H;
+    const int nch = (T + BC - 1) / BC;
+    float *ck = a.ckpt + (size_t)bh * nch * D * D;
+    const size_t soff = (size_t)bh * D * D;
+    const int col = tid % D, rb = tid / D;   // column and row block (or value block) of this thread
+    auto gidx = [&](int t, int c) -> size_t { return ((size_t)(b * T + t) * H + h) * D + c; };
+
+    // ---------------------------------------------------------------- helpers
+    auto load_tile = [&](float *dst, const void *src, int t0) {
+        for (int idx = tid; idx < BC * D; idx += BNT) {
+            const int i = idx / D, c = idx % D;
+            dst[i * LD + c] = t0 + i < T ? to_f32(((const IO *)src)[gidx(t0 + i, c)]) : 0.0f;
+        }
+    };
+    auto load_state = [&](float *dst, const float *src) {
+        for (int idx = tid; idx < D * D / 4; idx += BNT) {
+            const int c = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
+            const float4 x = src ? *(const float4 *)(src + (size_t)c * D + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            *(float4 *)(dst + c * LD + j4) = x;
+        }
+    };
+    auto store_state = [&](float *dst, const float *src) {
+        for (int idx = tid; idx < D * D / 4; idx += BNT) {
+            const int c = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
+            *(float4 *)(dst + (size_t)c * D + j4) = *(const float4 *)(src + c * LD + j4);
+        }
+    };
+    // G = inclusive cumsum of g over the chunk (in place), G_C, and the decayed q / k tiles
+    auto gates = [&](bool with_q) {
+        if (tid < D) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < BC; ++i) {
+                acc += Gs[i * LD + tid];
+                Gs[i * LD + tid] = acc;
+            }
+            GCs[tid] = acc;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < BC * D; idx += BNT) {
+            const int i = idx / D, c = idx % D;
+            const float G = Gs[i * LD + c], kv = Ks[i * LD + c];
+            const float e = __expf(G);
+            KHs[i * LD + c] = kv * e;
+            KTs[i * LD + c] = kv * __expf(GCs[c] - G);
+            if (with_q) QHs[i * LD + c] = Qs[i * LD + c] * e;
+        }
+    };
+    // Abar (j < i) and, with_p, P (j <= i): one warp per pair, lanes over channels
+    auto pair_dots = [&](bool with_p) {
+        for (int p = warp; p < BC * (BC + 1) / 2; p += BNT / 32) {
+            int i = 0;
+            while ((i + 1) * (i + 2) / 2 <= p) ++i;
+            const int j = p - i * (i + 1) / 2;
+            if (!with_p && j == i) continue;
+            float pv = 0.0f, av = 0.0f;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) {
+                const int c = lane + 32 * e;
+                const float x = Ks[j * LD + c] * __expf(Gs[i * LD + c] - Gs[j * LD + c]);
+                if (with_p) pv += Qs[i * LD + c] * x;
+                av += Ks[i * LD + c] * x;
+            }
+            pv = warp_sum(pv);
+            av = warp_sum(av);
+            if (lane == 0) {
+                if (with_p) Ps[i * CL + j] = pv;
+                if (j < i) ABs[i * CL + j] = av;
+            }
+        }
+    };
+    // M = (I + Diag(beta) Abar)^-1 by forward substitution; lane j owns column j (warp 0)
+    auto invert = [&]() {
+        if (lane < BC) {
+            const int j = lane;
+            float m[BC];
+#pragma unroll
+            for (int i = 0; i < BC; ++i) {
+                float s = 0.0f;
+#pragma unroll
+                for (int r = 0; r < i; ++r)
+                    if (r >= j) s += ABs[i * CL + r] * m[r];
+                m[i] = i < j ? 0.0f : (i == j ? 1.0f : -BETA[i] * s);
+            }
+#pragma unroll
+            for (int i = 0; i < BC; ++i) Ms[i * CL + j] = m[i];
+        }
+    };
+    // X = V - K^ S in place in Vs; (row block, column) partition
+    auto ks_x = [&]() {
+        float acc[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) acc[r] = 0.0f;
+        for (int c = 0; c < D; c += 4) {
+            const float s0 = Ss[(c + 0) * LD + col], s1 = Ss[(c + 1) * LD + col];
+            const float s2 = Ss[(c + 2) * LD + col], s3 = Ss[(c + 3) * LD + col];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const float4 kh = *(const float4 *)(KHs + (rb * RPT + r) * LD + c);
+                acc[r] += kh.x * s0 + kh.y * s1 + kh.z * s2 + kh.w * s3;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) Vs[(rb * RPT + r) * LD + col] -= acc[r];
+    };
+    // U = M (beta X)
+    auto u_from_x = [&]() {
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int i = rb * RPT + r;
+            float acc = 0.0f;
+            for (int m = 0; m <= i; ++m) acc += Ms[i * CL + m] * BETA[m] * Vs[m * LD + col];
+            Us[i * LD + col] = acc;
+        }
+    };
+
+    // ---------------------------------------------------------------- forward sweep: checkpoints
+    load_state(Ss, a.s0 ? a.s0 + soff : nullptr);
+    __syncthreads();
+    for (int n = 0; n < nch; ++n) {
+        const int t0 = n * BC;
+        store_state(ck + (size_t)n * D * D, Ss);
+        load_tile(Ks, a.k, t0);
+        load_tile(Gs, a.g, t0);
+        load_tile(Vs, a.v, t0);
+        if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
+        __syncthreads();
+        gates(false);
+        pair_dots(false);
+        __syncthreads();
+        if (warp == 0) invert();
+        ks_x();
+        __syncthreads();
+        u_from_x();
+        __syncthreads();
+        // S <- Diag(exp G_C) S + K~^T U; (column, value block) partition
+        {
+            const float gc = __expf(GCs[col]);
+            float acc[JPT];
+#pragma unroll
+            for (int jj = 0; jj < JPT; ++jj) acc[jj] = gc * Ss[col * LD + rb * JPT + jj];
+            for (int i = 0; i < BC; ++i) {
+                const float kt = KTs[i * LD + col];
+#pragma unroll
+                for (int jj = 0; jj < JPT; jj += 4) {
+                    const float4 u = *(const float4 *)(Us + i * LD + rb * JPT + jj);
+                    acc[jj] += kt * u.x; acc[jj + 1] += kt * u.y; acc[jj + 2] += kt * u.z; acc[jj + 3] += kt * u.w;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < JPT; ++jj) Ss[col * LD + rb * JPT + jj] = acc[jj];
+        }
+        __syncthreads();
+    }
+
+    // ---------------------------------------------------------------- reverse sweep
+    load_state(dSs, a.dST ? a.dST + soff : nullptr);
+    for (int n = nch - 1; n >= 0; --n) {
+        const int t0 = n * BC;
+        load_state(Ss, ck + (size_t)n * D * D);
+        load_tile(Qs, a.q, t0);
+        load_tile(Ks, a.k, t0);
+        load_tile(Gs, a.g, t0);
+        load_tile(Vs, a.v, t0);
+        load_tile(dOs, a.dO, t0);
+        if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
+        __syncthreads();
+        gates(true);
+        pair_dots(true);
+        __syncthreads();
+        if (warp == 0) invert();
+        ks_x();
+        __syncthreads();
+        u_from_x();
+        __syncthreads();
+
+        // dU = P^T dO + K~ dS_next, (row block, column) partition; then per (row, channel):
+        // dq <- exp(G) dO S^T, dk- <- exp(G_C - G) U dS_next^T and its share of dG_C
+        float dq[RPT], dkp[RPT], dkm[RPT];
+        {
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const int m = rb * RPT + r;
+                float acc = 0.0f;
+                for (int i = m; i < BC; ++i) acc += Ps[i * CL + m] * dOs[i * LD + col];
+                dUs[m * LD + col] = acc;
+            }
+            float acc[RPT];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) acc[r] = 0.0f;
+            for (int c = 0; c < D; c += 4) {
+                const float s0 = dSs[(c + 0) * LD + col], s1 = dSs[(c + 1) * LD + col];
+                const float s2 = dSs[(c + 2) * LD + col], s3 = dSs[(c + 3) * LD + col];
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const float4 kt = *(const float4 *)(KTs + (rb * RPT + r) * LD + c);
+                    acc[r] += kt.x * s0 + kt.y * s1 + kt.z * s2 + kt.w * s3;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) dUs[(rb * RPT + r) * LD + col] += acc[r];
+        }
+        {
+            const int c = col;
+            float aq[RPT], aw[RPT];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) aq[r] = aw[r] = 0.0f;
+            for (int j = 0; j < D; j += 4) {
+                const float4 s = *(const float4 *)(Ss + c * LD + j);
+                const float4 ds = *(const float4 *)(dSs + c * LD + j);
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const int i = rb * RPT + r;
+                    const float4 o = *(const float4 *)(dOs + i * LD + j);
+                    const float4 u = *(const float4 *)(Us + i * LD + j);
+                    aq[r] += o.x * s.x + o.y * s.y + o.z * s.z + o.w * s.w;
+                    aw[r] += u.x * ds.x + u.y * ds.y + u.z * ds.z + u.w * ds.w;
+                }
+            }
+            float kpart = 0.0f;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const int i = rb * RPT + r;
+                const float G = Gs[i * LD + c];
+                dq[r] = __expf(G) * aq[r];
+                dkm[r] = __expf(GCs[c] - G) * aw[r];
+                kpart += Ks[i * LD + c] * dkm[r];
+            }
+            REDK[rb * D + c] = kpart;
+        }
+        __syncthreads();
+        // dZ = M^T dU, into the K~ tile (free now)
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int m = rb * RPT + r;
+            float acc = 0.0f;
+            for (int i = m; i < BC; ++i) acc += Ms[i * CL + m] * dUs[i * LD + col];
+            KTs[m * LD + col] = acc;
+        }
+        __syncthreads();
+        // dP (j <= i), dA (j < i) and rowsum(dZ . X): one warp per dot, lanes over columns
+        for (int p = warp; p < BC * (BC + 1) + BC; p += BNT / 32) {
+            int kind, i, j;
+            if (p < BC * (BC + 1) / 2) {
+                kind = 0; i = 0;
+                while ((i + 1) * (i + 2) / 2 <= p) ++i;
+                j = p - i * (i + 1) / 2;
+            } else if (p < BC * (BC + 1)) {
+                kind = 1; const int pp = p - BC * (BC + 1) / 2; i = 0;
+                while ((i + 1) * (i + 2) / 2 <= pp) ++i;
+                j = pp - i * (i + 1) / 2;
+                if (j == i) continue;   // dA is strictly lower
+            } else {
+                kind = 2; i = j = p - BC * (BC + 1);
+            }
+            const float *x = kind == 0 ? dOs + i * LD : KTs + i * LD;
+            const float *y = kind == 0 ? Us + j * LD : (kind == 1 ? Us + j * LD : Vs + j * LD);
+            float s = 0.0f;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) s += x[lane + 32 * e] * y[lane + 32 * e];
+            s = warp_sum(s);
+            if (lane == 0) {
+                if (kind == 0) dPs[i * CL + j] = s;
+                else if (kind == 1) dAs[i * CL + j] = -s;
+                else DBETA[i] = s;
+            }
+        }
+        __syncthreads();
+        // dbeta += rowsum(dA . Abar), dAbar = Diag(beta) dA (warp 0, lane = row);
+        // dX = Diag(beta) dZ in place (everyone)
+        if (warp == 0 && lane < BC) {
+            const int i = lane;
+            float s = 0.0f;
+            for (int j = 0; j < i; ++j) {
+                const float d = dAs[i * CL + j];
+                s += d * ABs[i * CL + j];
+                dAs[i * CL + j] = BETA[i] * d;
+            }
+            DBETA[i] += s;
+        }
+        for (int idx = tid; idx < BC * D; idx += BNT) {
+            const int i = idx / D, c = idx % D;
+            KTs[i * LD + c] *= BETA[i];
+        }
+        __syncthreads();
+        // per (row, channel): dk+ <- -exp(G) dX S^T, the pairwise terms, dG; then per
+        // (channel, value block): dS <- Diag(exp G_C) dS + Q^^T dO - K^^T dX and the decay
+        // share of dG_C
+        {
+            const int c = col;
+            float ax[RPT];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) ax[r] = 0.0f;
+            for (int j = 0; j < D; j += 4) {
+                const float4 s = *(const float4 *)(Ss + c * LD + j);
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    const float4 x = *(const float4 *)(KTs + (rb * RPT + r) * LD + j);
+                    ax[r] += x.x * s.x + x.y * s.y + x.z * s.z + x.w * s.w;
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const int i = rb * RPT + r;
+                const float Gi = Gs[i * LD + c], qi = Qs[i * LD + c], ki = Ks[i * LD + c];
+                float aq = dq[r], ap = -__expf(Gi) * ax[r], am = dkm[r];
+                for (int j = 0; j <= i; ++j) {
+                    const float e = __expf(Gi - Gs[j * LD + c]) * Ks[j * LD + c];
+                    aq += dPs[i * CL + j] * e;
+                    if (j < i) ap += dAs[i * CL + j] * e;
+                }
+                for (int m = i; m < BC; ++m) {
+                    const float e = __expf(Gs[m * LD + c] - Gi);
+                    float w = dPs[m * CL + i] * Qs[m * LD + c];
+                    if (m > i) w += dAs[m * CL + i] * Ks[m * LD + c];
+                    am += w * e;
+                }
+                dq[r] = aq;
+                dkp[r] = ap;
+                dkm[r] = am;
+                dUs[i * LD + c] = qi * aq + ki * ap - ki * am;   // dG (dU is consumed)
+                if (t0 + i < T) {
+                    ((IO *)a.dq)[gidx(t0 + i, c)] = from_f32<IO>(aq);
+                    ((IO *)a.dk)[gidx(t0 + i, c)] = from_f32<IO>(ap + am);
+                }
+            }
+        }
+        {
+            const float gc = __expf(GCs[col]);
+            float acc[JPT];
+            float dec = 0.0f;
+#pragma unroll
+            for (int jj = 0; jj < JPT; ++jj) {
+                const float ds = dSs[col * LD + rb * JPT + jj];
+                dec += ds * Ss[col * LD + rb * JPT + jj];
+                acc[jj] = gc * ds;
+            }
+            REDS[rb * D + col] = gc * dec;
+            for (int i = 0; i < BC; ++i) {
+                const float qh = QHs[i * LD + col], kh = KHs[i * LD + col];
+#pragma unroll
+                for (int jj = 0; jj < JPT; jj += 4) {
+                    const float4 o = *(const float4 *)(dOs + i * LD + rb * JPT + jj);
+                    const float4 x = *(const float4 *)(KTs + i * LD + rb * JPT + jj);
+                    acc[jj] += qh * o.x - kh * x.x; acc[jj + 1] += qh * o.y - kh * x.y;
+                    acc[jj + 2] += qh * o.z - kh * x.z; acc[jj + 3] += qh * o.w - kh * x.w;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < JPT; ++jj) dSs[col * LD + rb * JPT + jj] = acc[jj];
+        }
+        __syncthreads();
+        // dg = reverse cumsum of dG, with dG_C added to the last row; dv = dX; dbeta
+        if (tid < D) {
+            float acc = 0.0f;
+#pragma unroll
+            for (int r = 0; r < NB; ++r) acc += REDK[r * D + tid] + REDS[r * D + tid];
+            for (int i = BC - 1; i >= 0; --i) {
+                acc += dUs[i * LD + tid];
+                if (t0 + i < T) ((IO *)a.dg)[gidx(t0 + i, tid)] = from_f32<IO>(acc);
+            }
+        }
+        for (int idx = tid; idx < BC * D; idx += BNT) {
+            const int i = idx / D, c = idx % D;
+            if (t0 + i < T) ((IO *)a.dv)[gidx(t0 + i, c)] = from_f32<IO>(KTs[i * LD + c]);
+        }
+        if (tid < BC && t0 + tid < T) ((IO *)a.dbeta)[(size_t)(b * T + t0 + tid) * H + h] = from_f32<IO>(DBETA[tid]);
+        __syncthreads();
+    }
+    if (a.ds0) store_state(a.ds0 + soff, dSs);
+}
+
+template <typename IO, int D>
+cudaError_t launch_bwd_t(const BwdArgs &a, int B, cudaStream_t s)
+{
+    static cudaError_t attr = cudaFuncSetAttribute(kda_backward_kernel<IO, D>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)BwdLayout<D>::BYTES);
+    if (attr != cudaSuccess) return attr;
+    kda_backward_kernel<IO, D><<<B * a.H, BNT, BwdLayout<D>::BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int T, int H, int d)
+{
+    const size_t nch = (size_t)(T + BC - 1) / BC;
+    return (size_t)B * H * nch * d * d * sizeof(float);
+}
+
+cudaError_t launch_backward(const BackwardArgs &x, cudaStream_t s)
+{
+    BwdArgs a{x.q, x.k, x.v, x.g, x.beta, x.s0, x.dO, x.dST, x.dq, x.dk, x.dv, x.dg, x.dbeta, x.ds0,
+              x.ckpt, x.T, x.H};
+    if (x.io == IO_F32) return x.d == 128 ? launch_bwd_t<float, 128>(a, x.B, s) : launch_bwd_t<float, 64>(a, x.B, s);
+    return x.d == 128 ? launch_bwd_t<__nv_bfloat16, 128>(a, x.B, s) : launch_bwd_t<__nv_bfloat16, 64>(a, x.B, s);
+}
+
+}  // namespace kda

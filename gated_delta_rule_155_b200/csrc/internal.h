@@ -83,4 +83,19 @@ cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueArgs &a, cudaStream_t s);
 cudaError_t launch_fill_state(const float *s0, float *sT, size_t n, cudaStream_t s);
 
+// Gradients of the recurrence (dk = dv = d).
+struct BackwardArgs {
+    const void *q, *k, *v, *g, *beta;   // io dtype, [B, T, H, d] / [B, T, H]
+    const float *s0;                    // nullable
+    const void *dO;                     // io dtype
+    const float *dST;                   // nullable
+    void *dq, *dk, *dv, *dg, *dbeta;    // io dtype
+    float *ds0;                         // nullable
+    float *ckpt;                        // backward_workspace_bytes()
+    int B, T, H, d;
+    IoType io;
+};
+size_t backward_workspace_bytes(int B, int T, int H, int d);
+cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
+
 }  // namespace kda

@@ -44,6 +44,10 @@ def _load():
     lib.kda_forward_chunked.argtypes = [vp] * 8 + [i] * 6 + [i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 4 + [i, vp]
+    lib.kda_backward_workspace_size.restype = i
+    lib.kda_backward_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
+    lib.kda_backward_chunked.restype = i
+    lib.kda_backward_chunked.argtypes = [vp] * 15 + [sz] + [i] * 5 + [i, vp]
     lib.kda_forward_chunked_varlen.restype = i
     lib.kda_forward_chunked_varlen.argtypes = [vp] * 9 + [i] * 6 + [i, vp]
     lib.kda_layer_workspace_size.restype = i
@@ -64,6 +68,7 @@ _lib = _load()
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_abi_version", "kda_forward_chunked",
                     "kda_decode_step", "kda_layer_workspace_size", "kda_layer_forward",
                     "kda_layer_forward_noalloc", "kda_layer_decode_step", "kda_forward_chunked_varlen",
+                    "kda_backward_workspace_size", "kda_backward_chunked",
                     "kda_check_device_error")
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES
@@ -161,6 +166,48 @@ def kda_forward_chunked_varlen(q, k, v, g, beta, cu_seqlens, initial_state=None,
                                            _stream(stream)),
            "kda_forward_chunked_varlen")
     return out, final_state
+
+
+def kda_backward_workspace_size(B, T, H, dk, dv, dtype):
+    n = ctypes.c_size_t(0)
+    _check(_lib.kda_backward_workspace_size(B, T, H, dk, dv, _io_code(dtype), ctypes.byref(n)),
+           "kda_backward_workspace_size")
+    return int(n.value)
+
+
+def kda_backward_chunked(q, k, v, g, beta, d_out, initial_state=None, d_final_state=None, *,
+                         grads=None, d_initial_state=None, workspace=None, stream=None):
+    """Gradients of kda_forward_chunked.  Returns dict dq, dk, dv, dg, dbeta (io dtype) and
+    d_initial_state (fp32 [B, H, dk, dv]).  ``grads`` may hold preallocated outputs;
+    ``workspace`` (uint8 CUDA tensor) is allocated with torch when not given."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = q.dtype
+    for t, s, n in ((q, (B, T, H, dk), "q"), (k, (B, T, H, dk), "k"), (g, (B, T, H, dk), "g"),
+                    (v, (B, T, H, dv), "v"), (beta, (B, T, H), "beta"), (d_out, (B, T, H, dv), "d_out")):
+        _need(t, s, io, n)
+    _need(initial_state, (B, H, dk, dv), torch.float32, "initial_state", allow_none=True)
+    _need(d_final_state, (B, H, dk, dv), torch.float32, "d_final_state", allow_none=True)
+    gr = dict(grads or {})
+    shapes = {"dq": (B, T, H, dk), "dk": (B, T, H, dk), "dg": (B, T, H, dk), "dv": (B, T, H, dv),
+              "dbeta": (B, T, H)}
+    for n, s in shapes.items():
+        if gr.get(n) is None:
+            gr[n] = torch.empty(s, dtype=io, device=q.device)
+        _need(gr[n], s, io, n)
+    if d_initial_state is None:
+        d_initial_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(d_initial_state, (B, H, dk, dv), torch.float32, "d_initial_state")
+    need = kda_backward_workspace_size(B, T, H, dk, dv, io)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.kda_backward_chunked(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(initial_state), _ptr(d_out), _ptr(d_final_state),
+        _ptr(gr["dq"]), _ptr(gr["dk"]), _ptr(gr["dv"]), _ptr(gr["dg"]), _ptr(gr["dbeta"]), _ptr(d_initial_state),
+        _ptr(workspace), ws_bytes, B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_backward_chunked")
+    gr["d_initial_state"] = d_initial_state
+    return gr
 
 
 def kda_decode_step(q, k, v, g, beta, state, out=None, *, stream=None):
@@ -299,6 +346,7 @@ def kda_check_device_error(stream=None):
 # short names
 forward_chunked = kda_forward_chunked
 forward_chunked_varlen = kda_forward_chunked_varlen
+backward_chunked = kda_backward_chunked
 decode_step = kda_decode_step
 layer_forward = kda_layer_forward
 layer_workspace_size = kda_layer_workspace_size

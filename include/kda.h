@@ -81,6 +81,40 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
                                  int chunk, kda_dtype_t io, kda_stream_t stream);
 
 /*
+ * Bytes of device workspace kda_backward_chunked needs: the fp32 state at the start of
+ * every 16-token chunk, B * H * ceil(T / 16) * dk * dv * 4.  dk must equal dv
+ * (KDA_ERR_UNSUPPORTED otherwise).  *bytes is written on KDA_OK.
+ */
+kda_status_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
+                                         size_t *bytes);
+
+/*
+ * kda_backward_chunked — gradients of the recurrence of kda_forward_chunked (training;
+ * the pages' runs differentiate the KDA layer: maxtext PR #5550, its jax.grad test and the
+ * C4 training steps).  Given d_out = dL/dout and d_final_state = dL/dS_T, writes dL/d of
+ * every input.  Computed in fp32 from the io-dtype inputs: a forward sweep stores the
+ * chunk-start states in `workspace`, then a reverse sweep over 16-token chunks recomputes
+ * each chunk and applies the chain rule (pairwise decays exp(G_i - G_j), j <= i, so no
+ * gate overflows).
+ *   q, k, g, v, beta, initial_state   as kda_forward_chunked (inputs, unchanged)
+ *   d_out          [B, T, H, dv] io dtype
+ *   d_final_state  [B, H, dk, dv] fp32 or NULL (zero)
+ *   d_q, d_k, d_g  [B, T, H, dk] io dtype (written; d_g is the gradient of the log-decay g)
+ *   d_v            [B, T, H, dv] io dtype (written)
+ *   d_beta         [B, T, H] io dtype (written)
+ *   d_initial_state [B, H, dk, dv] fp32 (written) or NULL; may equal d_final_state
+ *   workspace      device buffer of kda_backward_workspace_size() bytes, 256-byte aligned
+ * Supported: dk = dv in {64, 128}, both dtypes.  T = 0: d_initial_state receives
+ * d_final_state (or zeros).
+ */
+kda_status_t kda_backward_chunked(const void *q, const void *k, const void *v, const void *g,
+                                  const void *beta, const float *initial_state, const void *d_out,
+                                  const float *d_final_state, void *d_q, void *d_k, void *d_v,
+                                  void *d_g, void *d_beta, float *d_initial_state, void *workspace,
+                                  size_t workspace_bytes, int B, int T, int H, int dk, int dv,
+                                  kda_dtype_t io, kda_stream_t stream);
+
+/*
  * kda_forward_chunked_varlen — chunked prefill of N packed sequences of different lengths
  * (the variable-length batches that segment ids or a padding mask describe; the MaxText
  * port of the Kimi-K3 model rejects packing for KDA).  Each sequence runs the recurrence

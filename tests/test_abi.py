@@ -96,6 +96,25 @@ def test_forward_chunked_varlen_rejects_bad_arguments(lib):
     assert call(s0=MIS) == 3
 
 
+def test_backward_rejects_bad_arguments(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.kda_backward_workspace_size(2, 33, 3, 128, 128, 1, ctypes.byref(n)) == 0
+    assert n.value == 2 * 3 * 3 * 128 * 128 * 4          # three 16-token chunks per head
+    assert lib.kda_backward_workspace_size(2, 33, 3, 128, 64, 1, ctypes.byref(n)) == 2
+
+    def call(q=A16, ws=A16, ws_bytes=1 << 40, dk=128, dv=128, T=33, dgp=A16):
+        return lib.kda_backward_chunked(q, A16, A16, A16, A16, None, A16, None, A16, A16, A16, dgp, A16, None,
+                                        ws, ws_bytes, 2, T, 3, dk, dv, 1, None)
+    assert call(q=None) == 1
+    assert call(dgp=None) == 1
+    assert call(T=-1) == 1
+    assert call(dk=128, dv=64) == 2
+    assert call(q=MIS) == 3
+    assert call(ws=None) == 6
+    assert call(ws_bytes=1024) == 6
+    assert call(ws=P(0x100010)) == 3
+
+
 def test_decode_rejects_bad_arguments(lib):
     args = [A16] * 7
     ok = lambda **kw: lib.kda_decode_step(*[kw.get(n, a) for n, a in zip("qkvgbso", args)],
