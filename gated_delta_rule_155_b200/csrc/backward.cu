@@ -33,6 +33,7 @@ namespace {
 
 constexpr int BC = 16;     // tokens per chunk
 constexpr int BNT = 512;   // threads per CTA
+static_assert(2 * BC * BC == BNT, "the dot phase maps a thread pair to each (i, j)");
 
 template <int D>
 struct BwdLayout {
@@ -49,6 +50,11 @@ struct BwdLayout {
     static constexpr int FLOATS = REDS + NB * D;
     static constexpr size_t BYTES = sizeof(float) * FLOATS;
 };
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u)
+{
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
 
 struct BwdArgs {
     const void *q, *k, *v, *g, *beta;   // io dtype
@@ -85,10 +91,61 @@ kda_backward_kernel(BwdArgs a)
     auto gidx = [&](int t, int c) -> size_t { return ((size_t)(b * T + t) * H + h) * D + c; };
 
     // ---------------------------------------------------------------- helpers
-    auto load_tile = [&](float *dst, const void *src, int t0) {
-        for (int idx = tid; idx < BC * D; idx += BNT) {
-            const int i = idx / D, c = idx % D;
-            dst[i * LD + c] = t0 + i < T ? to_f32(((const IO *)src)[gidx(t0 + i, c)]) : 0.0f;
+    // A chunk's tiles (and, when given, a state) in 16-byte pieces: every thread issues all of
+    // its loads before it stores any, so the chunk pays one memory latency, not one per piece.
+    constexpr int EPC = 16 / (int)sizeof(IO);          // elements per 16-byte piece
+    constexpr int PPT = BC * D / EPC;                  // pieces per tile
+    // the tile pointers are chosen by a compare chain, so they stay in registers
+    auto pick = [](auto const *arr, int n, int tl) {
+        auto r = arr[0];
+#pragma unroll
+        for (int x = 1; x < 5; ++x)
+            if (x < n && tl == x) r = arr[x];
+        return r;
+    };
+    auto load_chunk = [&](float *const *dst, const void *const *src, int ntiles, int t0, float *sdst,
+                          const float *ssrc) {
+        constexpr int MAXP = (5 * PPT + BNT - 1) / BNT;
+        constexpr int SP = D * D / 4 / BNT;            // state float4s per thread
+        uint4 raw[MAXP];
+        float4 st[SP];
+        if (sdst) {
+#pragma unroll
+            for (int e = 0; e < SP; ++e) {
+                const int idx = tid + BNT * e, c = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
+                st[e] = ssrc ? *(const float4 *)(ssrc + (size_t)c * D + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < MAXP; ++e) {
+            const int f = tid + BNT * e, tl = f / PPT, pc = f % PPT;
+            const int i = pc / (D / EPC), c = (pc % (D / EPC)) * EPC;
+            raw[e] = make_uint4(0u, 0u, 0u, 0u);
+            if (tl < ntiles && t0 + i < T) raw[e] = *(const uint4 *)((const IO *)pick(src, ntiles, tl) + gidx(t0 + i, c));
+        }
+        if (sdst) {
+#pragma unroll
+            for (int e = 0; e < SP; ++e) {
+                const int idx = tid + BNT * e, c = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
+                *(float4 *)(sdst + c * LD + j4) = st[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < MAXP; ++e) {
+            const int f = tid + BNT * e, tl = f / PPT, pc = f % PPT;
+            const int i = pc / (D / EPC), c = (pc % (D / EPC)) * EPC;
+            if (tl < ntiles) {
+                float *o = pick(dst, ntiles, tl) + i * LD + c;
+                if constexpr (sizeof(IO) == 2) {
+                    const float2 x0 = bf16x2_to_float2(raw[e].x), x1 = bf16x2_to_float2(raw[e].y);
+                    const float2 x2 = bf16x2_to_float2(raw[e].z), x3 = bf16x2_to_float2(raw[e].w);
+                    *(float4 *)o = make_float4(x0.x, x0.y, x1.x, x1.y);
+                    *(float4 *)(o + 4) = make_float4(x2.x, x2.y, x3.x, x3.y);
+                } else {
+                    *(float4 *)o = make_float4(__uint_as_float(raw[e].x), __uint_as_float(raw[e].y),
+                                               __uint_as_float(raw[e].z), __uint_as_float(raw[e].w));
+                }
+            }
         }
     };
     auto load_state = [&](float *dst, const float *src) {
@@ -199,9 +256,11 @@ kda_backward_kernel(BwdArgs a)
     for (int n = 0; n < nch; ++n) {
         const int t0 = n * BC;
         store_state(ck + (size_t)n * D * D, Ss);
-        load_tile(Ks, a.k, t0);
-        load_tile(Gs, a.g, t0);
-        load_tile(Vs, a.v, t0);
+        {
+            float *const dst[3] = {Ks, Gs, Vs};
+            const void *const src[3] = {a.k, a.g, a.v};
+            load_chunk(dst, src, 3, t0, nullptr, nullptr);
+        }
         if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         gates(false);
@@ -217,7 +276,10 @@ kda_backward_kernel(BwdArgs a)
             const float gc = __expf(GCs[col]);
             float acc[JPT];
 #pragma unroll
-            for (int jj = 0; jj < JPT; ++jj) acc[jj] = gc * Ss[col * LD + rb * JPT + jj];
+            for (int jj = 0; jj < JPT; jj += 4) {
+                const float4 x = *(const float4 *)(Ss + col * LD + rb * JPT + jj);
+                acc[jj] = gc * x.x; acc[jj + 1] = gc * x.y; acc[jj + 2] = gc * x.z; acc[jj + 3] = gc * x.w;
+            }
             for (int i = 0; i < BC; ++i) {
                 const float kt = KTs[i * LD + col];
 #pragma unroll
@@ -227,7 +289,8 @@ kda_backward_kernel(BwdArgs a)
                 }
             }
 #pragma unroll
-            for (int jj = 0; jj < JPT; ++jj) Ss[col * LD + rb * JPT + jj] = acc[jj];
+            for (int jj = 0; jj < JPT; jj += 4)
+                *(float4 *)(Ss + col * LD + rb * JPT + jj) = make_float4(acc[jj], acc[jj + 1], acc[jj + 2], acc[jj + 3]);
         }
         __syncthreads();
     }
@@ -236,12 +299,11 @@ kda_backward_kernel(BwdArgs a)
     load_state(dSs, a.dST ? a.dST + soff : nullptr);
     for (int n = nch - 1; n >= 0; --n) {
         const int t0 = n * BC;
-        load_state(Ss, ck + (size_t)n * D * D);
-        load_tile(Qs, a.q, t0);
-        load_tile(Ks, a.k, t0);
-        load_tile(Gs, a.g, t0);
-        load_tile(Vs, a.v, t0);
-        load_tile(dOs, a.dO, t0);
+        {
+            float *const dst[5] = {Qs, Ks, Gs, Vs, dOs};
+            const void *const src[5] = {a.q, a.k, a.g, a.v, a.dO};
+            load_chunk(dst, src, 5, t0, Ss, ck + (size_t)n * D * D);
+        }
         if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         gates(true);
@@ -317,31 +379,31 @@ kda_backward_kernel(BwdArgs a)
             KTs[m * LD + col] = acc;
         }
         __syncthreads();
-        // dP (j <= i), dA (j < i) and rowsum(dZ . X): one warp per dot, lanes over columns
-        for (int p = warp; p < BC * (BC + 1) + BC; p += BNT / 32) {
-            int kind, i, j;
-            if (p < BC * (BC + 1) / 2) {
-                kind = 0; i = 0;
-                while ((i + 1) * (i + 2) / 2 <= p) ++i;
-                j = p - i * (i + 1) / 2;
-            } else if (p < BC * (BC + 1)) {
-                kind = 1; const int pp = p - BC * (BC + 1) / 2; i = 0;
-                while ((i + 1) * (i + 2) / 2 <= pp) ++i;
-                j = pp - i * (i + 1) / 2;
-                if (j == i) continue;   // dA is strictly lower
-            } else {
-                kind = 2; i = j = p - BC * (BC + 1);
+        // dP (j <= i), dA (j < i) and rowsum(dZ . X): a thread pair per (i, j), each thread
+        // summing one half of the columns
+        {
+            const int o = tid >> 1, hf = tid & 1, i = o / BC, j = o % BC;
+            const float *xo = dOs + i * LD + hf * (D / 2), *xz = KTs + i * LD + hf * (D / 2);
+            const float *yu = Us + j * LD + hf * (D / 2), *yx = Vs + i * LD + hf * (D / 2);
+            float sp = 0.0f, sa = 0.0f, sb = 0.0f;
+#pragma unroll 4
+            for (int c = 0; c < D / 2; c += 4) {
+                const float4 u = *(const float4 *)(yu + c), x = *(const float4 *)(xo + c);
+                const float4 z = *(const float4 *)(xz + c);
+                sp += x.x * u.x + x.y * u.y + x.z * u.z + x.w * u.w;
+                sa += z.x * u.x + z.y * u.y + z.z * u.z + z.w * u.w;
+                if (i == j) {
+                    const float4 v = *(const float4 *)(yx + c);
+                    sb += z.x * v.x + z.y * v.y + z.z * v.z + z.w * v.w;
+                }
             }
-            const float *x = kind == 0 ? dOs + i * LD : KTs + i * LD;
-            const float *y = kind == 0 ? Us + j * LD : (kind == 1 ? Us + j * LD : Vs + j * LD);
-            float s = 0.0f;
-#pragma unroll
-            for (int e = 0; e < D / 32; ++e) s += x[lane + 32 * e] * y[lane + 32 * e];
-            s = warp_sum(s);
-            if (lane == 0) {
-                if (kind == 0) dPs[i * CL + j] = s;
-                else if (kind == 1) dAs[i * CL + j] = -s;
-                else DBETA[i] = s;
+            sp += __shfl_xor_sync(0xffffffffu, sp, 1);
+            sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+            sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+            if (hf == 0) {
+                if (j <= i) dPs[i * CL + j] = sp;
+                if (j < i) dAs[i * CL + j] = -sa;
+                if (i == j) DBETA[i] = sb;
             }
         }
         __syncthreads();
@@ -409,10 +471,11 @@ kda_backward_kernel(BwdArgs a)
             float acc[JPT];
             float dec = 0.0f;
 #pragma unroll
-            for (int jj = 0; jj < JPT; ++jj) {
-                const float ds = dSs[col * LD + rb * JPT + jj];
-                dec += ds * Ss[col * LD + rb * JPT + jj];
-                acc[jj] = gc * ds;
+            for (int jj = 0; jj < JPT; jj += 4) {
+                const float4 ds = *(const float4 *)(dSs + col * LD + rb * JPT + jj);
+                const float4 sv = *(const float4 *)(Ss + col * LD + rb * JPT + jj);
+                dec += ds.x * sv.x + ds.y * sv.y + ds.z * sv.z + ds.w * sv.w;
+                acc[jj] = gc * ds.x; acc[jj + 1] = gc * ds.y; acc[jj + 2] = gc * ds.z; acc[jj + 3] = gc * ds.w;
             }
             REDS[rb * D + col] = gc * dec;
             for (int i = 0; i < BC; ++i) {
@@ -426,7 +489,8 @@ kda_backward_kernel(BwdArgs a)
                 }
             }
 #pragma unroll
-            for (int jj = 0; jj < JPT; ++jj) dSs[col * LD + rb * JPT + jj] = acc[jj];
+            for (int jj = 0; jj < JPT; jj += 4)
+                *(float4 *)(dSs + col * LD + rb * JPT + jj) = make_float4(acc[jj], acc[jj + 1], acc[jj + 2], acc[jj + 3]);
         }
         __syncthreads();
         // dg = reverse cumsum of dG, with dG_C added to the last row; dv = dX; dbeta
