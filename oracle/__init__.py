@@ -153,6 +153,32 @@ def recurrent_varlen(q, k, v, g, beta, cu_seqlens, s0=None, *, nthreads=0):
     return o, sT
 
 
+def layer_varlen(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
+                 o_gate_raw, cu_seqlens, o_norm_w=None, *, s0=None, **kw):
+    """The layer core over N packed sequences, each run by ``layer`` on its own tokens (so the
+    conv history and the state start fresh at every sequence).  Token-major inputs
+    ([T_total, H*dk], [T_total, H, dk], ...); s0 [N, H, dk, dv] or None.
+    Returns (out [T_total, H, dv], S_T [N, H, dk, dv])."""
+    cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
+    N = len(cu) - 1
+    Tt, H, dk = np.shape(g_raw)
+    dv = np.shape(o_gate_raw)[-1]
+    out = np.zeros((Tt, H, dv))
+    sT = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        a, b = cu[n], cu[n + 1]
+        s_n = None if s0 is None else _f64(s0)[n:n + 1]
+        if b == a:
+            sT[n] = 0.0 if s_n is None else s_n[0]
+            continue
+        o, st = layer(*(_f64(x)[None, a:b] for x in (q_raw, k_raw, v_raw)), conv_q, conv_k, conv_v,
+                      _f64(g_raw)[None, a:b], A_log, dt_bias, _f64(b_raw)[None, a:b], _f64(o_gate_raw)[None, a:b],
+                      o_norm_w, s0=s_n, **kw)
+        out[a:b] = o[0]
+        sT[n] = st[0]
+    return out, sT
+
+
 def decode(q, k, v, g, beta, state, *, nthreads=0):
     """One decode step.  q, k, g: [B, H, dk]; v: [B, H, dv]; beta: [B, H];
     state: [B, H, dk, dv].  Returns (o [B, H, dv], new_state) — the input is not modified."""

@@ -530,6 +530,48 @@ def test_layer_gate_bound_zero_equals_vanishing_decay_rate():
     assert np.max(np.abs(o5 - o4)) > 1e-3
 
 
+def _layer_raw(rng, T, H, d):
+    return dict(q_raw=rng.standard_normal((T, H * d)), k_raw=rng.standard_normal((T, H * d)),
+                v_raw=rng.standard_normal((T, H * d)), g_raw=rng.standard_normal((T, H, d)),
+                b_raw=rng.standard_normal((T, H)), o_gate_raw=rng.standard_normal((T, H, d)))
+
+
+def test_layer_varlen_equal_lengths_equal_the_batched_layer():
+    rng = np.random.default_rng(34)
+    B, T, H, d = 3, 7, 2, 4
+    r = _layer_raw(rng, B * T, H, d)
+    ws = [rng.standard_normal((H * d, 4)) * 0.5 for _ in range(3)]
+    A = rng.uniform(0, 1, H)
+    s0 = rng.standard_normal((B, H, d, d)) * 0.1
+    ub = lambda x: x.reshape((B, T) + x.shape[1:])
+    ob, sb = oracle.layer(ub(r["q_raw"]), ub(r["k_raw"]), ub(r["v_raw"]), *ws, ub(r["g_raw"]), A, None,
+                          ub(r["b_raw"]), ub(r["o_gate_raw"]), None, io_bf16=False, s0=s0)
+    ov, sv = oracle.layer_varlen(r["q_raw"], r["k_raw"], r["v_raw"], *ws, r["g_raw"], A, None, r["b_raw"],
+                                 r["o_gate_raw"], np.arange(B + 1) * T, None, s0=s0, io_bf16=False)
+    np.testing.assert_array_equal(ov, ob.reshape(ov.shape))
+    np.testing.assert_array_equal(sv, sb)
+
+
+def test_layer_varlen_conv_does_not_cross_sequences():
+    """Changing the last raw tokens of one sequence leaves the next sequence's outputs
+    unchanged (its conv history starts from zeros) and changes its own."""
+    rng = np.random.default_rng(35)
+    H, d = 2, 4
+    cu = np.array([0, 5, 11, 11, 14])
+    r = _layer_raw(rng, 14, H, d)
+    ws = [rng.standard_normal((H * d, 4)) * 0.5 for _ in range(3)]
+    A = rng.uniform(0, 1, H)
+    o1, _ = oracle.layer_varlen(*(r[n] for n in ("q_raw", "k_raw", "v_raw")), *ws, r["g_raw"], A, None,
+                                r["b_raw"], r["o_gate_raw"], cu, io_bf16=False)
+    r2 = {n: x.copy() for n, x in r.items()}
+    for n in ("q_raw", "k_raw", "v_raw"):
+        r2[n][3:5] += 1.0
+    o2, _ = oracle.layer_varlen(*(r2[n] for n in ("q_raw", "k_raw", "v_raw")), *ws, r2["g_raw"], A, None,
+                                r2["b_raw"], r2["o_gate_raw"], cu, io_bf16=False)
+    np.testing.assert_array_equal(o1[5:], o2[5:])
+    assert np.max(np.abs(o1[3:5] - o2[3:5])) > 1e-3
+
+
 def test_layer_conv_is_causal_per_channel():
     """Changing raw inputs at token t changes no layer output before t."""
     rng = np.random.default_rng(26)
