@@ -74,6 +74,46 @@ kda_status_t check_dims(int B, int T, int H, int dk, int dv, kda_dtype_t io)
     return KDA_OK;
 }
 
+// The layer core for B sequences of T tokens, or (cu != nullptr) for B packed sequences
+// with offsets cu over a token axis of T rows; dims already checked.
+kda_status_t layer_core(const void *q_raw, const void *k_raw, const void *v_raw, const float *conv_q,
+                        const float *conv_k, const float *conv_v, const void *g_raw, const float *A_log,
+                        const float *dt_bias, float gate_lower_bound, const void *b_raw, const void *o_gate_raw,
+                        const float *o_norm_w, float norm_eps, const float *initial_state, void *out,
+                        float *final_state, void *workspace, size_t workspace_bytes, int B, int T, int H, int dk,
+                        int dv, kda_dtype_t io, kda_stream_t stream, const int *cu)
+{
+    if (!(norm_eps >= 0.0f) || !(gate_lower_bound <= 0.0f)) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !g_raw ||
+                  !A_log || !b_raw || !o_gate_raw || !out))
+        return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,
+                          b_raw, o_gate_raw, o_norm_w, initial_state, out, final_state};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (T == 0) return cuda_status(kda::launch_fill_state(initial_state, final_state,
+                                                          (size_t)B * H * dk * dv, s));
+    const int rows = cu ? 1 : B;   // batch rows of the token-major tensors
+    const LayerWorkspace w = layer_workspace(rows, T, H, dk, dv);
+    if (!workspace || workspace_bytes < w.total) return KDA_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255u) != 0) return KDA_ERR_MISALIGNED;
+    char *ws = (char *)workspace;
+    float *wq = (float *)(ws + w.q), *wk = (float *)(ws + w.k), *wv = (float *)(ws + w.v);
+    float *wg = (float *)(ws + w.g), *wb = (float *)(ws + w.beta), *wo = (float *)(ws + w.o);
+
+    kda::PrologueArgs pa{q_raw, k_raw, v_raw, g_raw, b_raw, conv_q, conv_k, conv_v, A_log, dt_bias,
+                         gate_lower_bound, wq, wk, wv, wg, wb, rows, T, H, dk, dv, io_of(io), cu, cu ? B : 0};
+    cudaError_t e = kda::launch_prologue(pa, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    kda::ChunkArgs ca{wq, wk, wv, wg, wb, initial_state, wo, final_state, B, T, H, dk, dv,
+                      kda::IO_F32, true, true, true, true, error_word(), cu};
+    e = kda::chunk_f32_supported(ca) ? kda::launch_chunk_f32(ca, s) : kda::launch_chunk_simt(ca, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    kda::EpilogueArgs ea{wo, o_gate_raw, o_norm_w, norm_eps, out, rows, T, H, dv, io_of(io)};
+    return cuda_status(kda::launch_epilogue(ea, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -215,34 +255,29 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
 {
     kda_status_t st = check_dims(B, T, H, dk, dv, io);
     if (st != KDA_OK) return st;
-    if (!(norm_eps >= 0.0f) || !(gate_lower_bound <= 0.0f)) return KDA_ERR_INVALID_ARG;
-    if (T > 0 && (!q_raw || !k_raw || !v_raw || !conv_q || !conv_k || !conv_v || !g_raw ||
-                  !A_log || !b_raw || !o_gate_raw || !out))
-        return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias,
-                          b_raw, o_gate_raw, o_norm_w, initial_state, out, final_state};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (T == 0) return cuda_status(kda::launch_fill_state(initial_state, final_state,
-                                                          (size_t)B * H * dk * dv, s));
-    const LayerWorkspace w = layer_workspace(B, T, H, dk, dv);
-    if (!workspace || workspace_bytes < w.total) return KDA_ERR_WORKSPACE;
-    if (((uintptr_t)workspace & 255u) != 0) return KDA_ERR_MISALIGNED;
-    char *ws = (char *)workspace;
-    float *wq = (float *)(ws + w.q), *wk = (float *)(ws + w.k), *wv = (float *)(ws + w.v);
-    float *wg = (float *)(ws + w.g), *wb = (float *)(ws + w.beta), *wo = (float *)(ws + w.o);
+    return layer_core(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, gate_lower_bound, b_raw,
+                      o_gate_raw, o_norm_w, norm_eps, initial_state, out, final_state, workspace, workspace_bytes, B,
+                      T, H, dk, dv, io, stream, nullptr);
+}
 
-    kda::PrologueArgs pa{q_raw, k_raw, v_raw, g_raw, b_raw, conv_q, conv_k, conv_v, A_log, dt_bias,
-                         gate_lower_bound, wq, wk, wv, wg, wb, B, T, H, dk, dv, io_of(io)};
-    cudaError_t e = kda::launch_prologue(pa, s);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
-    kda::ChunkArgs ca{wq, wk, wv, wg, wb, initial_state, wo, final_state, B, T, H, dk, dv,
-                      kda::IO_F32, true, true, true, true, error_word()};
-    e = kda::chunk_f32_supported(ca) ? kda::launch_chunk_f32(ca, s) : kda::launch_chunk_simt(ca, s);
-    if (e != cudaSuccess) return KDA_ERR_CUDA;
-    kda::EpilogueArgs ea{wo, o_gate_raw, o_norm_w, norm_eps, out, B, T, H, dv, io_of(io)};
-    return cuda_status(kda::launch_epilogue(ea, s));
+kda_status_t kda_layer_forward_varlen(const void *q_raw, const void *k_raw, const void *v_raw,
+                                      const float *conv_q, const float *conv_k, const float *conv_v,
+                                      const void *g_raw, const float *A_log, const float *dt_bias,
+                                      float gate_lower_bound, const void *b_raw, const void *o_gate_raw,
+                                      const float *o_norm_w, float norm_eps, const float *initial_state,
+                                      void *out, float *final_state, const int *cu_seqlens, void *workspace,
+                                      size_t workspace_bytes, int N, int T_total, int H, int dk, int dv,
+                                      kda_dtype_t io, kda_stream_t stream)
+{
+    kda_status_t st = check_dims(1, T_total, H, dk, dv, io);
+    if (st != KDA_OK) return st;
+    if (N < 1) return KDA_ERR_INVALID_ARG;
+    if ((long long)N * H > INT32_MAX / 2) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(cu_seqlens)) return KDA_ERR_MISALIGNED;
+    return layer_core(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, gate_lower_bound, b_raw,
+                      o_gate_raw, o_norm_w, norm_eps, initial_state, out, final_state, workspace, workspace_bytes, N,
+                      T_total, H, dk, dv, io, stream, cu_seqlens);
 }
 
 kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const void *v_raw,

@@ -39,6 +39,8 @@ struct PrologueArgs {
     float *q, *k, *v, *g, *beta;  // workspace outputs, fp32
     int B, T, H, dk, dv;
     IoType io;
+    const int *cu = nullptr;      // packed sequences: offsets [nseq + 1], device (B = 1, T = total)
+    int nseq = 0;
 };
 
 struct EpilogueArgs {

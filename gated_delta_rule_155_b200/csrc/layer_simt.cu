@@ -53,13 +53,33 @@ template <int N> KDA_DEVICE void stn(float *p, const float (&v)[N])
     else *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
 }
 
+// Where the run starting at token t0 sits among packed sequences: lo = first token of its
+// sequence (the conv's history floor), nb = first token of the next sequence, si = its index.
+// Fixed length: lo = 0, nb = no boundary.  Offsets are clamped into the array, so malformed
+// ones cannot send a read out of bounds.
+struct SeqPos {
+    int lo, nb, si;
+};
+KDA_DEVICE SeqPos seq_pos(const int *cu, int nseq, int t0)
+{
+    if (!cu) return SeqPos{0, 0x7fffffff, 0};
+    int a = 0, b = nseq - 1;   // the last sequence whose start is <= t0
+    while (a < b) {
+        const int m = (a + b + 1) >> 1;
+        if (cu[m] <= t0) a = m;
+        else b = m - 1;
+    }
+    return SeqPos{cu[a], cu[a + 1], a};
+}
+
 // One head's channels of one input stream over a run of tokens t0 .. t0 + nt - 1: causal
 // depthwise conv (PyTorch Conv1d tap order: y[t, c] = sum_i w[c, i] x[t - 3 + i, c], zero
-// history) + SiLU [+ L2-norm over the head's D channels].  Lane l owns channels
-// N l .. N l + N - 1 and slides a three-row window, so every input row is read once.
+// history before each sequence's first token) + SiLU [+ L2-norm over the head's D channels].
+// Lane l owns channels N l .. N l + N - 1 and slides a three-row window, so every input row is
+// read once; the window restarts from zeros where a packed sequence begins.
 template <typename IO, int D, bool NORM>
 KDA_DEVICE void conv_stream(const IO *__restrict__ x, size_t rs, const float *__restrict__ w, float *__restrict__ dst,
-                            size_t drs, int t0, int nt, int lane)
+                            size_t drs, int t0, int nt, int lane, SeqPos sp, const int *cu, int nseq)
 {
     constexpr int N = D / 32;
     const int c0 = N * lane;
@@ -70,11 +90,17 @@ KDA_DEVICE void conv_stream(const IO *__restrict__ x, size_t rs, const float *__
         wt[e][0] = wv.x; wt[e][1] = wv.y; wt[e][2] = wv.z; wt[e][3] = wv.w;
         x3[e] = x2[e] = x1[e] = 0.0f;
     }
-    if (t0 >= 3) ldn<N>(x + (size_t)(t0 - 3) * rs + c0, x3);
-    if (t0 >= 2) ldn<N>(x + (size_t)(t0 - 2) * rs + c0, x2);
-    if (t0 >= 1) ldn<N>(x + (size_t)(t0 - 1) * rs + c0, x1);
+    if (t0 - 3 >= sp.lo) ldn<N>(x + (size_t)(t0 - 3) * rs + c0, x3);
+    if (t0 - 2 >= sp.lo) ldn<N>(x + (size_t)(t0 - 2) * rs + c0, x2);
+    if (t0 - 1 >= sp.lo) ldn<N>(x + (size_t)(t0 - 1) * rs + c0, x1);
     for (int r = 0; r < nt; ++r) {
         const int t = t0 + r;
+        while (t >= sp.nb) {   // a packed sequence starts here (empty ones are stepped over)
+#pragma unroll
+            for (int e = 0; e < N; ++e) x3[e] = x2[e] = x1[e] = 0.0f;
+            ++sp.si;
+            sp.nb = sp.si < nseq ? cu[sp.si + 1] : 0x7fffffff;
+        }
         float xt[N], y[N];
         ldn<N>(x + (size_t)t * rs + c0, xt);
         float ss = 0.0f;
@@ -113,13 +139,14 @@ kda_prologue_kernel(PrologueArgs a)
     const int nt = min(RUN, a.T - t0);
     const size_t rsk = (size_t)a.H * DK, rsv = (size_t)a.H * DV;
     const size_t bt0 = (size_t)b * a.T;   // first (b, t) row of this sequence
+    const SeqPos sp = seq_pos(a.cu, a.nseq, t0);
 
     conv_stream<IO, DK, true>((const IO *)a.q_raw + bt0 * rsk + (size_t)h * DK, rsk, a.conv_q + (size_t)h * DK * 4,
-                              a.q + (bt0 * a.H + h) * DK, rsk, t0, nt, lane);
+                              a.q + (bt0 * a.H + h) * DK, rsk, t0, nt, lane, sp, a.cu, a.nseq);
     conv_stream<IO, DK, true>((const IO *)a.k_raw + bt0 * rsk + (size_t)h * DK, rsk, a.conv_k + (size_t)h * DK * 4,
-                              a.k + (bt0 * a.H + h) * DK, rsk, t0, nt, lane);
+                              a.k + (bt0 * a.H + h) * DK, rsk, t0, nt, lane, sp, a.cu, a.nseq);
     conv_stream<IO, DV, false>((const IO *)a.v_raw + bt0 * rsv + (size_t)h * DV, rsv, a.conv_v + (size_t)h * DV * 4,
-                               a.v + (bt0 * a.H + h) * DV, rsv, t0, nt, lane);
+                               a.v + (bt0 * a.H + h) * DV, rsv, t0, nt, lane, sp, a.cu, a.nseq);
     // gate g = max(-exp(A_log[h]) softplus(g_raw + dt_bias[h, c]), lb) and beta = sigmoid(b_raw)
     {
         constexpr int N = DK / 32;

@@ -44,6 +44,8 @@ def _load():
     lib.kda_forward_chunked.argtypes = [vp] * 8 + [i] * 6 + [i, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 4 + [i, vp]
+    lib.kda_layer_forward_varlen.restype = i
+    lib.kda_layer_forward_varlen.argtypes = [vp] * 9 + [f] + [vp] * 3 + [f] + [vp] * 5 + [sz] + [i] * 5 + [i, vp]
     lib.kda_backward_workspace_size.restype = i
     lib.kda_backward_workspace_size.argtypes = [i] * 6 + [ctypes.POINTER(sz)]
     lib.kda_backward_chunked.restype = i
@@ -68,7 +70,7 @@ _lib = _load()
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_abi_version", "kda_forward_chunked",
                     "kda_decode_step", "kda_layer_workspace_size", "kda_layer_forward",
                     "kda_layer_forward_noalloc", "kda_layer_decode_step", "kda_forward_chunked_varlen",
-                    "kda_backward_workspace_size", "kda_backward_chunked",
+                    "kda_backward_workspace_size", "kda_backward_chunked", "kda_layer_forward_varlen",
                     "kda_check_device_error")
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES
@@ -272,6 +274,45 @@ def kda_layer_forward(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log,
         _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _lb(gate_lower_bound), _ptr(b_raw), _ptr(o_gate_raw),
         _ptr(o_norm_w), float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(workspace),
         ws_bytes, B, T, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward")
+    return out, final_state
+
+
+def kda_layer_forward_varlen(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw, A_log, dt_bias, b_raw,
+                             o_gate_raw, cu_seqlens, o_norm_w=None, *, norm_eps=1e-6, initial_state=None,
+                             out=None, final_state=None, workspace=None, gate_lower_bound=None, stream=None):
+    """The layer core over N packed sequences.  q_raw, k_raw: [T_total, H*dk]; v_raw: [T_total, H*dv];
+    g_raw: [T_total, H, dk]; b_raw: [T_total, H]; o_gate_raw: [T_total, H, dv]; cu_seqlens: int32 CUDA
+    [N + 1]; states [N, H, dk, dv].  Returns (out [T_total, H, dv], final_state)."""
+    Tt, H, dk = g_raw.shape
+    dv = o_gate_raw.shape[-1]
+    io = g_raw.dtype
+    f32 = torch.float32
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a 1-D tensor of N + 1 >= 2 offsets")
+    N = cu_seqlens.numel() - 1
+    _need(cu_seqlens, (N + 1,), torch.int32, "cu_seqlens")
+    for t, s, d, n in ((q_raw, (Tt, H * dk), io, "q_raw"), (k_raw, (Tt, H * dk), io, "k_raw"),
+                       (v_raw, (Tt, H * dv), io, "v_raw"), (b_raw, (Tt, H), io, "b_raw"),
+                       (o_gate_raw, (Tt, H, dv), io, "o_gate_raw"),
+                       (conv_q, (H * dk, 4), f32, "conv_q"), (conv_k, (H * dk, 4), f32, "conv_k"),
+                       (conv_v, (H * dv, 4), f32, "conv_v"), (A_log, (H,), f32, "A_log")):
+        _need(t, s, d, n)
+    _need(dt_bias, (H * dk,), f32, "dt_bias", allow_none=True)
+    _need(o_norm_w, (dv,), f32, "o_norm_w", allow_none=True)
+    _need(initial_state, (N, H, dk, dv), f32, "initial_state", allow_none=True)
+    _need(final_state, (N, H, dk, dv), f32, "final_state", allow_none=True)
+    if out is None:
+        out = torch.empty((Tt, H, dv), dtype=io, device=g_raw.device)
+    _need(out, (Tt, H, dv), io, "out")
+    need = kda_layer_workspace_size(1, Tt, H, dk, dv, io)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=g_raw.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.kda_layer_forward_varlen(
+        _ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(conv_q), _ptr(conv_k), _ptr(conv_v),
+        _ptr(g_raw), _ptr(A_log), _ptr(dt_bias), _lb(gate_lower_bound), _ptr(b_raw), _ptr(o_gate_raw),
+        _ptr(o_norm_w), float(norm_eps), _ptr(initial_state), _ptr(out), _ptr(final_state), _ptr(cu_seqlens),
+        _ptr(workspace), ws_bytes, N, Tt, H, dk, dv, _io_code(io), _stream(stream)), "kda_layer_forward_varlen")
     return out, final_state
 
 

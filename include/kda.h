@@ -192,6 +192,24 @@ kda_status_t kda_layer_forward(const void *q_raw, const void *k_raw, const void 
                                int B, int T, int H, int dk, int dv, kda_dtype_t io,
                                kda_stream_t stream);
 
+/*
+ * kda_layer_forward_varlen — kda_layer_forward over N packed sequences of different lengths
+ * (the padding-mask / segment-id case; see kda_forward_chunked_varlen).  Every raw tensor is
+ * token-major over T_total tokens ([T_total, H*dk], [T_total, H, dk], [T_total, H], ...);
+ * states are [N, H, dk, dv]; cu_seqlens is the device int32 [N + 1] offsets array (same
+ * rules as kda_forward_chunked_varlen).  The short conv's history is zero before each
+ * sequence's first token, so no input of one sequence reaches another's outputs.
+ * Workspace: kda_layer_workspace_size(1, T_total, H, dk, dv, io) bytes.
+ */
+kda_status_t kda_layer_forward_varlen(const void *q_raw, const void *k_raw, const void *v_raw,
+                                      const float *conv_q, const float *conv_k, const float *conv_v,
+                                      const void *g_raw, const float *A_log, const float *dt_bias,
+                                      float gate_lower_bound, const void *b_raw, const void *o_gate_raw,
+                                      const float *o_norm_w, float norm_eps, const float *initial_state,
+                                      void *out, float *final_state, const int *cu_seqlens, void *workspace,
+                                      size_t workspace_bytes, int N, int T_total, int H, int dk, int dv,
+                                      kda_dtype_t io, kda_stream_t stream);
+
 /* Size in bytes of the built-in scratch that kda_layer_forward_noalloc uses (64 MiB). */
 #define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

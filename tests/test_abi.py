@@ -171,6 +171,18 @@ def test_layer_workspace_and_argument_checks(lib):
     assert layer(ws=P(0x100010)) == 3  # workspace must be 256-byte aligned
 
 
+def test_layer_varlen_rejects_bad_arguments(lib):
+    def call(cu=A16, q=A16, N=3, Tt=100, eps=1e-6):
+        return lib.kda_layer_forward_varlen(q, A16, A16, A16, A16, A16, A16, A16, None, ctypes.c_float(-5.0),
+                                            A16, A16, None, ctypes.c_float(eps), None, A16, None, cu, A16, 1 << 40,
+                                            N, Tt, 2, 128, 128, 1, None)
+    assert call(cu=None) == 1
+    assert call(q=None) == 1
+    assert call(N=0) == 1
+    assert call(eps=-1.0) == 1
+    assert call(cu=MIS) == 3
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     """The binding raises at import when libkda.so is missing — there is no fallback."""
     import importlib.util

@@ -534,6 +534,57 @@ def test_layer_workload_B2_T16384_H96_sampled_heads(kda):
     check_heads(out, sT, ro, rs, heads, torch.bfloat16, roundings=2)
 
 
+def packed_layer_inputs(lens, H, d, io, seed, s0_std=0.05):
+    """Token-major layer inputs over sum(lens) tokens, their offsets and a per-sequence S_0."""
+    L = inputs.layer_inputs(1, int(sum(lens)), H, d, d, io=io, seed=seed, dt_bias_std=0.4, gain_std=0.2)
+    P = {n: (v[0] if n in ("q_raw", "k_raw", "v_raw", "g_raw", "b_raw", "o_gate_raw") else v) for n, v in L.items()}
+    P["cu_seqlens"] = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    P["s0"] = torch.randn((len(lens), H, d, d), generator=torch.Generator().manual_seed(seed)) * s0_std
+    return P
+
+
+def run_layer_varlen(kda, P, lb=None):
+    dev = "cuda"
+    to = lambda x: None if x is None else x.contiguous().to(dev)
+    N, H, d = P["s0"].shape[0], P["g_raw"].shape[1], P["g_raw"].shape[2]
+    sT = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    out, sT = kda.kda_layer_forward_varlen(
+        to(P["q_raw"]), to(P["k_raw"]), to(P["v_raw"]), to(P["conv_q"]), to(P["conv_k"]), to(P["conv_v"]),
+        to(P["g_raw"]), to(P["A_log"]), to(P["dt_bias"]), to(P["b_raw"]), to(P["o_gate_raw"]),
+        to(P["cu_seqlens"]), to(P["o_norm_w"]), initial_state=to(P["s0"]), final_state=sT, gate_lower_bound=lb)
+    kda.kda_check_device_error()
+    return out, sT
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d_", [64, 128])
+def test_layer_varlen_ragged(kda, io, d_):
+    """Packed sequences shorter than the conv (1, 2 tokens), shorter than a prologue run,
+    around a chunk and several chunks long, with empty ones between: every output and every
+    final state against the oracle run per sequence."""
+    lens = [0, 1, 2, 5, 63, 64, 0, 65, 7, 130]
+    P = packed_layer_inputs(lens, 3, d_, "f32" if io == torch.float32 else "bf16", seed=140 + d_)
+    out, sT = run_layer_varlen(kda, P, lb=-6.0)
+    a = {n: (None if v is None else f64(v)) for n, v in P.items()}
+    ro, rs = oracle.layer_varlen(a["q_raw"], a["k_raw"], a["v_raw"], a["conv_q"], a["conv_k"], a["conv_v"],
+                                 a["g_raw"], a["A_log"], a["dt_bias"], a["b_raw"], a["o_gate_raw"],
+                                 P["cu_seqlens"].numpy(), a["o_norm_w"], s0=a["s0"],
+                                 io_bf16=io == torch.bfloat16, gate_lower_bound=-6.0)
+    assert err(f64(out), ro, io, stored_bf16=2) <= tol(io)
+    assert serr(f64(sT), rs, io) <= 1.0
+
+
+def test_layer_varlen_equal_lengths_equal_the_batched_layer(kda):
+    """Three packed sequences of 70 tokens give kda_layer_forward's B = 3 results bit for bit."""
+    P = packed_layer_inputs([70, 70, 70], 2, 128, "bf16", seed=150)
+    ov, sv = run_layer_varlen(kda, P)
+    d = {n: (v.reshape((3, 70) + tuple(v.shape[1:])) if n in ("q_raw", "k_raw", "v_raw", "g_raw", "b_raw",
+                                                               "o_gate_raw") else v) for n, v in P.items()}
+    ob, sb = run_layer(kda, d)
+    assert torch.equal(ov.reshape(ob.shape), ob)
+    assert torch.equal(sv, sb)
+
+
 def test_layer_zero_gate_input_halves_output(kda):
     """o_gate_raw = 0: the output is exactly half the gain-scaled normalised output of the
     same call with a saturated gate (sigmoid(0) = 1/2)."""
