@@ -316,8 +316,8 @@ def run_ours(args):
                         f"H={Hv} dk=dv=128 bf16, zero initial state",
             "value": round(aggregate_rate(Tt, ms_v, ws), 1), "unit": "tokens/s", "ms_per_step": round(ms_v, 4),
             "roofline": {"bound": "hbm", "achieved": round(ach_v, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(ach_v / pk["hbm_gbs"], 4), "traffic": traffic_for("kda_chunk_tc"),
-                         "kernel": "kda_chunk_tc", "launch_ms": round(lms_v, 4), "bytes_per_launch": bytes_v}}
+                         "frac": round(ach_v / pk["hbm_gbs"], 4), "traffic": traffic_for("kda_chunk_tc_packed"),
+                         "kernel": "kda_chunk_tc (packed)", "launch_ms": round(lms_v, 4), "bytes_per_launch": bytes_v}}
         launches_per["varlen"] = 1
         del xv, ov, sv, dl
         torch.cuda.empty_cache()

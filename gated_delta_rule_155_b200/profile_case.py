@@ -3,6 +3,8 @@
     python -m gated_delta_rule_155_b200.profile_case prefill --B 2 --T 4096 --H 96 --launches 3
     python -m gated_delta_rule_155_b200.profile_case decode  --B 64 --H 96 --launches 3
     python -m gated_delta_rule_155_b200.profile_case layer   --B 1 --T 4096 --H 96 --launches 2
+    python -m gated_delta_rule_155_b200.profile_case varlen  --T 8192 --H 96 --launches 3
+    python -m gated_delta_rule_155_b200.profile_case backward --B 1 --T 1024 --H 148 --launches 2
 
 Inputs come from the seeded generators; nothing is checked or timed here (use the
 tests for parity and bench.py for timing).  Sizes should keep the inputs larger than
@@ -18,7 +20,7 @@ import torch
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode", "layer"])
+    ap.add_argument("kind", choices=["prefill", "decode", "layer", "varlen", "backward"])
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--H", type=int, default=96)
@@ -44,6 +46,21 @@ def main(argv=None):
         x = {n: dd["steps"][0][n].to(dev) for n in ("q", "k", "v", "g", "beta")}
         for _ in range(a.launches):
             kda.kda_decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], st)
+    elif a.kind == "varlen":
+        # packed sequences of 1..4096 tokens, a.T tokens in all (the packed workload's law)
+        lens = inputs.packed_lengths(a.T, 4096, 5)
+        dl = inputs.varlen_inputs(lens, a.H, a.d, a.d, io="bf16", seed=5)
+        x = [dl[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+        cu = dl["cu_seqlens"].to(dev)
+        sT = torch.empty((len(lens), a.H, a.d, a.d), device=dev)
+        for _ in range(a.launches):
+            kda.kda_forward_chunked_varlen(*x, cu, None, None, sT)
+    elif a.kind == "backward":
+        d = inputs.prefill_inputs(a.B, a.T, a.H, a.d, a.d, io="bf16", seed=2)
+        x = [d[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
+        dO = torch.randn(x[2].shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16).to(dev)
+        for _ in range(a.launches):
+            kda.kda_backward_chunked(*x, dO)
     else:
         L = inputs.layer_inputs(a.B, a.T, a.H, a.d, a.d, io="bf16", seed=4)
         to = lambda t: None if t is None else t.to(dev)
