@@ -132,7 +132,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_abi_version(void) { return 101; }
+int kda_abi_version(void) { return 102; }
 
 kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *initial_state, void *out,

@@ -516,9 +516,8 @@ kda_backward_kernel(BwdArgs a)
 template <typename IO, int D>
 cudaError_t launch_bwd_t(const BwdArgs &a, int B, cudaStream_t s)
 {
-    static cudaError_t attr = cudaFuncSetAttribute(kda_backward_kernel<IO, D>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)BwdLayout<D>::BYTES);
+    struct Tag;
+    const cudaError_t attr = smem_opt_in<Tag>((const void *)kda_backward_kernel<IO, D>, (int)BwdLayout<D>::BYTES);
     if (attr != cudaSuccess) return attr;
     kda_backward_kernel<IO, D><<<B * a.H, BNT, BwdLayout<D>::BYTES, s>>>(a);
     return cudaGetLastError();

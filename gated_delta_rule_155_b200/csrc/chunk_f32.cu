@@ -461,8 +461,8 @@ bool chunk_f32_supported(const ChunkArgs &a)
 
 cudaError_t launch_chunk_f32(const ChunkArgs &a, cudaStream_t s)
 {
-    static cudaError_t attr = cudaFuncSetAttribute(kda_chunk_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)F32_SMEM);
+    struct Tag;
+    const cudaError_t attr = smem_opt_in<Tag>((const void *)kda_chunk_f32_kernel, (int)F32_SMEM);
     if (attr != cudaSuccess) return attr;
     dim3 grid((unsigned)(a.B * a.H), 2u);
     kda_chunk_f32_kernel<<<grid, FNT, F32_SMEM, s>>>((const float *)a.q, (const float *)a.k, (const float *)a.v,

@@ -957,15 +957,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
         !make_map(&mv, a.v, mb, a.T, a.H) || !make_map(&mg, a.g, mb, a.T, a.H) ||
         !make_map(&mo, a.out, mb, a.T, a.H))
         return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(kda_chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SMEM_BYTES);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            SMEM_BYTES);
-    });
+    struct TagFixed;
+    struct TagPacked;
+    cudaError_t attr_err = smem_opt_in<TagFixed>((const void *)kda_chunk_tc_kernel<false>, SMEM_BYTES);
+    if (attr_err == cudaSuccess) attr_err = smem_opt_in<TagPacked>((const void *)kda_chunk_tc_kernel<true>, SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
     TcParams p{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
                (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err, a.cu};

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include <mutex>
+
 namespace kda {
 
 enum IoType { IO_F32 = 0, IO_BF16 = 1 };
@@ -84,6 +86,22 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueArgs &a, cudaStream_t s);
 cudaError_t launch_fill_state(const float *s0, float *sT, size_t n, cudaStream_t s);
+
+// Opts `fn` into `bytes` of dynamic shared memory on the current device.  The attribute
+// belongs to the device's context, so it is set once per device (a process may drive
+// several GPUs); Tag makes the flags distinct per kernel.
+constexpr int kMaxSmemDevices = 64;
+template <typename Tag>
+cudaError_t smem_opt_in(const void *fn, int bytes)
+{
+    static std::once_flag once[kMaxSmemDevices];
+    static cudaError_t err[kMaxSmemDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    if (dev < 0 || dev >= kMaxSmemDevices) return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    std::call_once(once[dev], [&] { err[dev] = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes); });
+    return err[dev];
+}
 
 // Gradients of the recurrence (dk = dv = d).
 struct BackwardArgs {

@@ -52,7 +52,7 @@ def test_status_strings(lib):
         s = lib.kda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.kda_status_string(99) == b"unknown status"
-    assert lib.kda_abi_version() == 101
+    assert lib.kda_abi_version() == 102
 
 
 P = ctypes.c_void_p
