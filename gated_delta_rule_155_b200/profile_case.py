@@ -5,6 +5,7 @@
     python -m gated_delta_rule_155_b200.profile_case layer   --B 1 --T 4096 --H 96 --launches 2
     python -m gated_delta_rule_155_b200.profile_case varlen  --T 8192 --H 96 --launches 3
     python -m gated_delta_rule_155_b200.profile_case backward --B 1 --T 1024 --H 148 --launches 2
+    python -m gated_delta_rule_155_b200.profile_case layer_decode --B 64 --H 96 --launches 3
 
 Inputs come from the seeded generators; nothing is checked or timed here (use the
 tests for parity and bench.py for timing).  Sizes should keep the inputs larger than
@@ -20,7 +21,7 @@ import torch
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("kind", choices=["prefill", "decode", "layer", "varlen", "backward"])
+    ap.add_argument("kind", choices=["prefill", "decode", "layer", "varlen", "backward", "layer_decode"])
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--T", type=int, default=4096)
     ap.add_argument("--H", type=int, default=96)
@@ -55,6 +56,17 @@ def main(argv=None):
         sT = torch.empty((len(lens), a.H, a.d, a.d), device=dev)
         for _ in range(a.launches):
             kda.kda_forward_chunked_varlen(*x, cu, None, None, sT)
+    elif a.kind == "layer_decode":
+        # one new token per sequence through the whole layer, conv caches and state in place
+        L = inputs.layer_inputs(a.B, 1, a.H, a.d, a.d, io="bf16", seed=3, conv_std=0.5, s0_std=0.02)
+        to = lambda t: None if t is None else t.contiguous().to(dev)
+        st = to(L["s0"])
+        caches = [torch.zeros((a.B, 3, a.H * a.d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        x = {n: to(L[n][:, 0]) for n in ("q_raw", "k_raw", "v_raw", "g_raw", "b_raw", "o_gate_raw")}
+        for _ in range(a.launches):
+            kda.kda_layer_decode_step(x["q_raw"], x["k_raw"], x["v_raw"], to(L["conv_q"]), to(L["conv_k"]),
+                                      to(L["conv_v"]), *caches, x["g_raw"], to(L["A_log"]), to(L["dt_bias"]),
+                                      x["b_raw"], x["o_gate_raw"], st, to(L["o_norm_w"]))
     elif a.kind == "backward":
         d = inputs.prefill_inputs(a.B, a.T, a.H, a.d, a.d, io="bf16", seed=2)
         x = [d[n].to(dev) for n in ("q", "k", "v", "g", "beta")]
