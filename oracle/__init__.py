@@ -42,25 +42,30 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def declare(lib):
+    """Set the argument types of every oracle entry point on a loaded copy of the C library
+    (the built one, or a test's deliberately mutated build of the same source)."""
+    i = ctypes.c_int
+    d = ctypes.c_double
+    sz = ctypes.c_size_t
+    lib.kda_oracle_recurrent.argtypes = [_dp] * 8 + [i] * 7
+    lib.kda_oracle_recurrent_backward.argtypes = [_dp] * 14 + [i] * 6
+    lib.kda_oracle_decode.argtypes = [_dp] * 7 + [i] * 5
+    lib.kda_oracle_short_conv_silu.argtypes = [_dp] * 3 + [i] * 5
+    lib.kda_oracle_l2norm.argtypes = [_dp, _dp, sz, i, d]
+    lib.kda_oracle_gate.argtypes = [_dp] * 3 + [d, _dp] + [i] * 4
+    lib.kda_oracle_sigmoid.argtypes = [_dp, _dp, sz]
+    lib.kda_oracle_out_norm_gate.argtypes = [_dp, _dp, _dp, d, i, _dp, sz, i]
+    lib.kda_oracle_layer.argtypes = [_dp] * 9 + [d] + [_dp] * 3 + [d, d, i, _dp, _dp, _dp] + [i] * 6
+    lib.kda_oracle_max_threads.restype = i
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            i = ctypes.c_int
-            d = ctypes.c_double
-            sz = ctypes.c_size_t
-            lib.kda_oracle_recurrent.argtypes = [_dp] * 8 + [i] * 7
-            lib.kda_oracle_recurrent_backward.argtypes = [_dp] * 14 + [i] * 6
-            lib.kda_oracle_decode.argtypes = [_dp] * 7 + [i] * 5
-            lib.kda_oracle_short_conv_silu.argtypes = [_dp] * 3 + [i] * 5
-            lib.kda_oracle_l2norm.argtypes = [_dp, _dp, sz, i, d]
-            lib.kda_oracle_gate.argtypes = [_dp] * 3 + [d, _dp] + [i] * 4
-            lib.kda_oracle_sigmoid.argtypes = [_dp, _dp, sz]
-            lib.kda_oracle_out_norm_gate.argtypes = [_dp, _dp, _dp, d, i, _dp, sz, i]
-            lib.kda_oracle_layer.argtypes = [_dp] * 9 + [d] + [_dp] * 3 + [d, d, i, _dp, _dp, _dp] + [i] * 6
-            lib.kda_oracle_max_threads.restype = i
-            _lib = lib
+            _lib = declare(ctypes.CDLL(build()))
     return _lib
 
 
