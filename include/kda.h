@@ -12,9 +12,21 @@
  * size between calls) and maxtext PR #5548's review, item 2 (KDA tensors A_log,
  * dt_bias, conv weights and o_norm kept in F32; exp(A_log) drives the decay).
  *
+ * Entry points
+ *   kda_forward_chunked          chunked prefill: outputs and final state
+ *   kda_forward_chunked_varlen   the same over N packed sequences (cu_seqlens)
+ *   kda_decode_step              one token per sequence, state in place
+ *   kda_layer_forward            the layer core (conv + SiLU, L2-norm, gate, beta,
+ *                                recurrence, RMSNorm x sigmoid gate); _noalloc and
+ *                                _varlen variants
+ *   kda_layer_decode_step        one decode step of the layer core with a conv cache
+ *   kda_backward_chunked         gradients of the recurrence's inputs
+ *   kda_*_workspace_size, kda_check_device_error, kda_status_string, kda_abi_version
+ *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless a comment says otherwise; the caller owns
- *     and allocates every buffer.  The library allocates no device memory.
+ *     and allocates every buffer.  The library allocates no device memory in any call
+ *     (kda_layer_forward_noalloc uses a fixed array the library holds from load time).
  *   - Layouts are dense and row-major (last index fastest):
  *       q, k, g : [B, T, H, dk]      v, out : [B, T, H, dv]      beta : [B, T, H]
  *       state   : [B, H, dk, dv] fp32
