@@ -111,6 +111,11 @@ def _need(t, shape, dtype, name, *, allow_none=False):
         raise ValueError(f"{name} is required")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    # the library launches on the current device, so every tensor must live there
+    cur = torch.cuda.current_device()
+    if t.device.index is not None and t.device.index != cur:
+        raise ValueError(f"{name} is on cuda:{t.device.index} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({t.device.index})")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if t.dtype != dtype:

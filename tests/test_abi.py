@@ -183,6 +183,24 @@ def test_layer_varlen_rejects_bad_arguments(lib):
     assert call(cu=MIS) == 3
 
 
+def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
+    """Kernels launch on the current device, so a tensor on another GPU is an error, caught
+    before any pointer reaches the library."""
+    import types
+
+    import torch
+
+    from gated_delta_rule_155_b200 import kda
+
+    fake = types.SimpleNamespace(is_cuda=True, device=types.SimpleNamespace(index=1), shape=(2, 3),
+                                 dtype=torch.float32, is_contiguous=lambda: True)
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current device is cuda:0"):
+        kda._need(fake, (2, 3), torch.float32, "q")
+    fake.device.index = 0
+    kda._need(fake, (2, 3), torch.float32, "q")        # same device: accepted
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     """The binding raises at import when libkda.so is missing — there is no fallback."""
     import importlib.util
