@@ -55,3 +55,17 @@ def test_one_bf16_rounding_of_the_update_operand_needs_the_rounding_term():
     rms = np.sqrt(np.mean(ref * ref))
     assert err.max() / (2e-2 * rms) > 1.2                                   # RMS-only bound fails
     assert np.max(err / (2e-2 * rms + 2.0 ** -8 * np.abs(ref))) < 0.9     # with the term it holds
+
+
+def test_storing_exact_outputs_in_bf16_needs_the_output_rounding_term():
+    """The exact fp64 outputs of 8 heads of the T = 4096 bf16 workload, merely rounded to
+    bf16 (what any bf16-output kernel must store), sit 1.9x above 2e-2 of the output RMS —
+    the outputs reach 17x their RMS — and within the bound once each element may be one bf16
+    rounding away, the term the output bound carries."""
+    d = inputs.prefill_inputs(1, 4096, 8, 128, 128, io="bf16", seed=1, s0_std=0.02)
+    o, _ = oracle.recurrent(*(d[n].double().numpy() for n in ("q", "k", "v", "g", "beta")),
+                            d["s0"].double().numpy())
+    err = np.abs(_bf16(o) - o)
+    rms = np.sqrt(np.mean(o * o))
+    assert err.max() / (2e-2 * rms) > 1.5
+    assert np.max(err / (2e-2 * rms + 2.0 ** -8 * np.abs(o))) < 0.8
