@@ -183,6 +183,30 @@ def test_layer_varlen_rejects_bad_arguments(lib):
     assert call(cu=MIS) == 3
 
 
+def header_prototypes():
+    """{name: number of parameters} of every function the header declares."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b(kda_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_declares_every_prototype_with_its_arity(lib):
+    """Each C entry point's ctypes declaration has as many arguments as its prototype in
+    include/kda.h, so a signature change cannot leave the binding behind."""
+    protos = header_prototypes()
+    assert len(protos) >= 13
+    for name, n in protos.items():
+        fn = getattr(lib, name)
+        if n == 0:
+            assert not fn.argtypes, f"{name} takes no arguments"
+            continue
+        assert fn.argtypes is not None, f"{name} has no argtypes in the binding"
+        assert len(fn.argtypes) == n, f"{name}: header has {n} parameters, binding {len(fn.argtypes)}"
+
+
 def test_binding_rejects_tensors_off_the_current_device(monkeypatch):
     """Kernels launch on the current device, so a tensor on another GPU is an error, caught
     before any pointer reaches the library."""
