@@ -1,9 +1,11 @@
 // api.cu — the C ABI of libkda.so (declared in include/kda.h).
 //
 // Every entry point validates all of its arguments before launching anything, so an
-// error status means nothing ran and no output was touched.  The library keeps no
-// state beyond one device error word per GPU (set by a kernel whose bounded wait
-// gave up) and allocates no device memory.
+// error status means nothing ran and no output was touched.  The library allocates no
+// device memory per call.  Its state: one device error word per GPU (set by a kernel
+// whose bounded wait gave up), the process-wide wait limit and failure injection of
+// kda_set_wait_test_hooks, and the KDA_NOALLOC_SCRATCH_BYTES array of noalloc.cu, which
+// every GPU that loads the library holds until exit.
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
@@ -74,6 +76,20 @@ kda_status_t check_dims(int B, int T, int H, int dk, int dv, kda_dtype_t io)
     return KDA_OK;
 }
 
+// One kernel per (dtype, head dims): bf16 at dk = dv = 128 runs on the tensor cores and
+// nowhere else — a device or driver that cannot run that kernel gets KDA_ERR_UNSUPPORTED,
+// not a slower kernel; fp32 at d = 128 runs the exact fp32 kernel; the other head-dim
+// pairs run the exact CUDA-core kernel.
+kda_status_t launch_chunked(const kda::ChunkArgs &a, cudaStream_t s)
+{
+    if (a.io == kda::IO_BF16 && a.dk == 128 && a.dv == 128) {
+        if (!kda::chunk_tc_supported(a)) return KDA_ERR_UNSUPPORTED;
+        return cuda_status(kda::launch_chunk_tc(a, s));
+    }
+    if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
+    return cuda_status(kda::launch_chunk_simt(a, s));
+}
+
 // The layer core for B sequences of T tokens, or (cu != nullptr) for B packed sequences
 // with offsets cu over a token axis of T rows; dims already checked.
 kda_status_t layer_core(const void *q_raw, const void *k_raw, const void *v_raw, const float *conv_q,
@@ -132,7 +148,7 @@ const char *kda_status_string(kda_status_t s)
     return "unknown status";
 }
 
-int kda_abi_version(void) { return 102; }
+int kda_abi_version(void) { return 103; }
 
 kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *initial_state, void *out,
@@ -151,9 +167,7 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
                                                           (size_t)B * H * dk * dv, s));
     kda::ChunkArgs a{q, k, v, g, beta, initial_state, out, final_state, B, T, H, dk, dv,
                      io_of(io), false, false, false, false, error_word()};
-    if (kda::chunk_tc_supported(a)) return cuda_status(kda::launch_chunk_tc(a, s));
-    if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
-    return cuda_status(kda::launch_chunk_simt(a, s));
+    return launch_chunked(a, s);
 }
 
 kda_status_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
@@ -215,9 +229,7 @@ kda_status_t kda_forward_chunked_varlen(const void *q, const void *k, const void
     // the kernels take B = N sequences over a token axis of T = T_total rows
     kda::ChunkArgs a{q, k, v, g, beta, initial_state, out, final_state, N, T_total, H, dk, dv,
                      io_of(io), false, false, false, false, error_word(), cu_seqlens};
-    if (kda::chunk_tc_supported(a)) return cuda_status(kda::launch_chunk_tc(a, s));
-    if (kda::chunk_f32_supported(a)) return cuda_status(kda::launch_chunk_f32(a, s));
-    return cuda_status(kda::launch_chunk_simt(a, s));
+    return launch_chunked(a, s);
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const void *g,
@@ -303,6 +315,12 @@ kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const v
                            g_raw, A_log, dt_bias, gate_lower_bound, b_raw, o_gate_raw, o_norm_w,
                            norm_eps, state, out, B, H, io_of(io)};
     return cuda_status(kda::launch_layer_decode(a, (cudaStream_t)stream));
+}
+
+kda_status_t kda_set_wait_test_hooks(unsigned long long wait_limit_ns, int skip_load_chunk)
+{
+    kda::set_wait_hooks(wait_limit_ns, skip_load_chunk);
+    return KDA_OK;
 }
 
 kda_status_t kda_check_device_error(kda_stream_t stream)

@@ -31,12 +31,13 @@
 // Precision.  bf16 operands alone would put errors of the order of one bf16 rounding
 // on top of the output's own bf16 rounding.  So the diagonal P[i][i] = q_i . k_i is
 // formed exactly in fp32 from the raw inputs, the diagonal 16x16 blocks of the Gram get a
-// second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U, Y and P enter their
+// second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U, Y, P and K~ enter their
 // products as hi + lo bf16 pairs (O += U_hi P_hi + U_lo P_hi + U_hi P_lo,
-// S += K~^T (U_hi + U_lo)), and the state is read at tf32 precision from its fp32 copy for
-// S^T Q^^T (Q^ kept in fp32).
+// S += K~_hi^T (U_hi + U_lo) + K~_lo^T U_hi), and the state is read at tf32 precision from
+// its fp32 copy for S^T Q^^T (Q^ kept in fp32).
 #include <cuda.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -59,6 +60,12 @@ constexpr int OFF_REG0 = 0;
 constexpr int OFF_REG1 = REG_BYTES;
 constexpr int ST_Q = 0, ST_K = 16384, ST_V = 32768, ST_G = 49152;     // inside a stage region
 constexpr int GR_R = 0, GR_CV = 32768;                                // inside a Gram region
+// K~ lo (bf16 MN-major, one 64-channel block per region): channel block cb lives at offset
+// ST_KLO of region cb, past the stage tiles.  In chunk n the stage region (n & 1) has that
+// tail free from the load onwards, so its block is written during prep; the other region's
+// tail holds Gram columns until the Gram MMA has run, so that block is kept in registers
+// across the Gram and written then.  Both are read by the state-update MMA at the chunk's end.
+constexpr int ST_KLO = 65536;
 constexpr int R_CB = 16384;                      // R: 128 rows x 128 B per channel block
 constexpr int CV_ROWS = 160, CV_CB = CV_ROWS * 128;
 // X1 (32 KB): Q^ in fp32 (tf32 K-major [i][c]), from prep until the O-init MMA (issued
@@ -94,6 +101,7 @@ constexpr int MS_PD = 832;                       // fp32 [4][64]: exact q_i . k_
 constexpr int MS_BAR = 1856;                     // uint64 [5]: tma0, tma1, mma, O init, Y
 constexpr int MS_TSLOT = 1896;                   // uint32
 constexpr int MS_ABORT = 1900;                   // int
+constexpr int MS_DRAIN = 1904;                   // uint64: MMA drain after an abort
 constexpr int MS_BRAW = 1920;                    // uint32 [2][64]: beta words in flight (cp.async)
 constexpr int MISC_BYTES = 2432;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
@@ -127,6 +135,8 @@ struct TcParams {
     int T, H;
     int *err;
     const int *cu;   // packed variable length: sequence offsets (null: fixed length T)
+    unsigned long long wait_ns;   // limit of each bounded mbarrier wait
+    int skip_load_chunk;          // failure injection: this chunk's tile load is never issued (-1: none)
 };
 
 KDA_DEVICE void unpack8(const uint4 &u, float (&f)[8])
@@ -164,6 +174,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *bar_y = bar_tma + 4;
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
+    uint64_t *bar_drain = (uint64_t *)(misc + MS_DRAIN);
     float *A32 = (float *)(sm + OFF_A32);
     float *LINV = (float *)(sm + OFF_LINV);
 
@@ -186,6 +197,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(bar_mma, 1);
         mbar_init(bar_o, 1);
         mbar_init(bar_y, 1);
+        mbar_init(bar_drain, 3);   // the three MMA-issuing threads
         *abort_flag = 0;
         for (int i = 0; i < 16; ++i) badmask[i] = 0u;
         fence_mbar_init();
@@ -201,7 +213,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
+    // Loads issued by thread 0 and loads consumed (uniform: counted after the barrier that
+    // follows the wait); after an abort at most one issued load has not been waited for.
+    int tma_issued = 0, tma_consumed = 0;
     auto issue_tma = [&](int n) {
+        if (n == p.skip_load_chunk) return;   // injected failure: the wait for it runs out
+        ++tma_issued;
         const int r = n & 1;
         uint8_t *st = sm + (r ? OFF_REG1 : OFF_REG0);
         const int t0 = tt0 + n * CK;
@@ -228,10 +245,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 
     uint32_t mma_phase = 0;
-    auto mma_wait = [&]() -> bool {
-        const bool ok = mbar_wait_bounded(bar_mma, mma_phase, abort_flag, p.err);
+    // A wait that gives up sets *abort_flag (and the device error word); every thread then
+    // leaves the chunk loop at the next check of the flag, each placed right after a block
+    // barrier and before any TMA or MMA issue, so the decision is the same for the whole CTA.
+    auto mma_wait = [&]() {
+        mbar_wait_bounded(bar_mma, mma_phase, abort_flag, p.err, p.wait_ns);
         mma_phase ^= 1u;
-        return ok;
     };
 
     constexpr uint32_t id_gram = idesc_bf16(128, CV_ROWS, false, false);
@@ -241,6 +260,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr uint32_t id_opn = idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t id_op = idesc_bf16(128, 64, false, false);
     constexpr uint32_t id_s = idesc_bf16(128, 128, false, true);
+    constexpr uint32_t id_s64 = idesc_bf16(128, 64, false, true);
 
     // beta of the next chunk is copied one chunk ahead, global -> shared by cp.async, so no
     // thread ever waits on its memory latency: the aligned 32-bit word that holds beta_t
@@ -265,7 +285,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint8_t *gro = sm + (X ? OFF_REG0 : OFF_REG1);
         const int t0 = n * CK;
 
-        if (!mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err)) break;
+        mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err, p.wait_ns);
 
         // ============================================================ prep
         if (tid < CK) {
@@ -330,6 +350,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncthreads();
+        if (*abort_flag) break;   // the wait for this chunk's tiles gave up
+        tma_consumed = n + 1;
         // pass B, one (block, channel) per thread: block log-decays L_J and the factors
         //   fG = exp(G_blockstart)      fL = exp(G_C - G_blockend)
         //   fM = exp(-L_B / 2) / SC     (block-start reference, 1 / SC, where L_B < BAD_LOG)
@@ -371,6 +393,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
         // from log-domain prefix sums, so no partial product can underflow; both are normal
         // numbers for block log-decays down to BAD_LOG (SC e^-168 ~ e^-84.8).
+        uint4 klo[2];   // this thread's K~ lo, two tokens x 8 channels of channel block cb
         {
 #pragma unroll
             for (int s = 0; s < 2; ++s) {
@@ -427,11 +450,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * gam[e];
                 *(uint4 *)(stg + ST_K + off) = pack8(o);
-                // K~ = exp(G_C - G_i) k (over g) = k (E2 / SC) fL
+                // K~ = exp(G_C - G_i) k = k (E2 / SC) fL: bf16 hi over g, bf16 residual to the
+                // K~ lo tile (now if this channel block's tail is free, else after the Gram)
                 ftab(FT_L + B, f);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
-                *(uint4 *)(stg + ST_G + off) = pack8(o);
+                {
+                    const uint4 hk = pack8(o);
+                    float hf[8], lo[8];
+                    unpack8(hk, hf);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
+                    *(uint4 *)(stg + ST_G + off) = hk;
+                    klo[s] = pack8(lo);
+                    if (cb == X) *(uint4 *)(stg + ST_KLO + swz(i, a)) = klo[s];
+                }
                 // Gram rows [Q_B; K_B] scaled by E1 fM = exp(G_i - m_B): hi part to the Gram
                 // rows, bf16 residual to X2 (free until the readback)
                 ftab(FT_M + B, f);
@@ -504,13 +537,14 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                        sdesc(sCVL + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_corr, 1);
             mma_commit(bar_mma);
         }
-        if (!mma_wait()) break;
+        mma_wait();
         tc_fence_after();
-        if (tid == 0 && n + 1 < nchunks) {
-            // the Gram region is free now; it was the stage of chunk n - 1, whose O tile must
-            // have been read out by its TMA store
-            bulk_wait_read_all();
-            issue_tma(n + 1);
+        if (cb != X) {
+            // the Gram MMA has read the other region's tail: this channel block's K~ lo goes there
+#pragma unroll
+            for (int s = 0; s < 2; ++s)
+                *(uint4 *)(gro + ST_KLO + swz(16 * (s == 0 ? pr : 3 - pr) + 8 * th + pp, a)) = klo[s];
+            fence_proxy_async();
         }
 
         // ============================================================ Gram readback -> P, A
@@ -605,6 +639,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncthreads();
+        if (*abort_flag) break;   // the Gram wait gave up
+        if (tid == 0 && n + 1 < nchunks) {
+            // the Gram region is free now; it was the stage of chunk n - 1, whose O tile must
+            // have been read out by its TMA store
+            bulk_wait_read_all();
+            issue_tma(n + 1);
+        }
         if (tid < 16) badmask[tid] = 0u;   // masks consumed
         // ============================================================ T (warps 0..7) || Y = K^ S (warps 8..15)
         // Warps 0..7 invert L = I + A and form T (named barrier 1).  Warps 8..15 (named barrier
@@ -754,7 +795,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                            id_op, 1);
                 mma_commit(bar_y);
             }
-            if (mbar_wait_bounded(bar_y, (uint32_t)(n & 1), abort_flag, p.err)) {
+            if (mbar_wait_bounded(bar_y, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns)) {
                 tc_fence_after();
                 // Y^T (fp32, tokens 32 hb .. 32 hb + 31) -> bf16 hi + lo
                 uint32_t r[32], hi[16], lo[16];
@@ -773,7 +814,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             // S^T <- S^T Diag(exp G_C): every reader of the chunk-start state is done once the
             // O init has completed (the split above and the Y MMAs read the copies)
-            if (mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err)) {
+            if (mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns)) {
                 tc_fence_after();
 #pragma unroll
                 for (int cc = 0; cc < 64; cc += 32) {
@@ -804,7 +845,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_ts(tmem + TM_U, tmem + TM_LO32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, 1);
             mma_commit(bar_mma);
         }
-        if (!mma_wait()) break;
+        mma_wait();
         tc_fence_after();
         {
             // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column; Y's are consumed)
@@ -824,9 +865,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         tc_fence_before();
         __syncthreads();
+        if (*abort_flag) break;   // the U wait gave up
         if (tid == 0) {
             tc_fence_after();
             const uint32_t sP = smem_u32(stg + ST_P), sPL = smem_u32(stg + ST_PL), sG = smem_u32(stg + ST_G);
+            const uint32_t sKL0 = smem_u32(sm + OFF_REG0 + ST_KLO), sKL1 = smem_u32(sm + OFF_REG1 + ST_KLO);
             for (int kk = 0; kk < 4; ++kk) {
                 mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
                 mma_ts(tmem + TM_O, tmem + TM_LO32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
@@ -835,10 +878,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int kk = 0; kk < 4; ++kk) {
                 mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
                 mma_ts(tmem + TM_S, tmem + TM_LO32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
+                // K~ lo, one 64-channel block (state columns) per MMA
+                mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sKL0 + kk * 2048, 8192, 1024), id_s64, 1);
+                mma_ts(tmem + TM_S + 64, tmem + TM_HI32 + kk * 8, sdesc(sKL1 + kk * 2048, 8192, 1024), id_s64, 1);
             }
             mma_commit(bar_mma);
         }
-        if (!mma_wait()) break;
+        mma_wait();
         tc_fence_after();
         {
             // O^T -> bf16 tile in the stage's V tile (dead since the U~ MMA; the load tiles'
@@ -857,6 +903,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (*abort_flag) break;   // the O / state wait gave up
         if (tail) {
             // the last chunk of a packed sequence: its tile's later rows are the next
             // sequence's, so only the valid rows are written, 16 bytes per thread and pass
@@ -884,6 +931,24 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int e = 0; e < 32; ++e) sT[(size_t)(32 * cg + e) * DD + v] = __uint_as_float(r[e]);
     }
+    if (*abort_flag) {
+        // A bounded wait gave up (the flag is read after a block barrier, so the whole CTA is
+        // here).  Everything asynchronous this CTA started finishes before its shared and tensor
+        // memory are released: the MMAs of the three issuing threads (one commit each on
+        // bar_drain), a tile load issued but not yet waited for, the beta copies and the bulk
+        // stores.  These operations were really issued, so they complete; the waits are
+        // bounded all the same.
+        constexpr unsigned long long DRAIN_NS = 2000000000ull;
+        if (tid == 0 || tid == 256 || tid == NT - 32) mma_commit(bar_drain);
+        if (tid == 0) {
+            if (tma_issued > tma_consumed) {
+                const int c = tma_consumed;
+                mbar_wait_timed(&bar_tma[c & 1], (uint32_t)((c >> 1) & 1), DRAIN_NS);
+            }
+            mbar_wait_timed(bar_drain, 0u, DRAIN_NS);
+        }
+    }
+    if (tid < CK) cp_async_wait_all();
     if (tid == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
@@ -945,8 +1010,22 @@ bool device_is_sm100()
 bool chunk_tc_supported(const ChunkArgs &a)
 {
     // beta is fetched as aligned 32-bit words (cp.async), so it must start on a 4-byte boundary
+    // (the entry points require 16)
     return a.io == IO_BF16 && a.dk == DD && a.dv == DD && !a.qkv_f32 && !a.g_f32 && !a.beta_f32 && !a.out_f32 &&
            a.T > 0 && ((uintptr_t)a.beta & 3) == 0 && device_is_sm100() && encode_fn() != nullptr;
+}
+
+namespace {
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_skip_load_chunk{-1};
+}  // namespace
+
+WaitHooks wait_hooks() { return WaitHooks{g_wait_ns.load(), g_skip_load_chunk.load()}; }
+
+void set_wait_hooks(unsigned long long wait_ns, int skip_load_chunk)
+{
+    g_wait_ns.store(wait_ns ? wait_ns : kDefaultWaitNs);
+    g_skip_load_chunk.store(skip_load_chunk < 0 ? -1 : skip_load_chunk);
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
@@ -962,8 +1041,10 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s)
     cudaError_t attr_err = smem_opt_in<TagFixed>((const void *)kda_chunk_tc_kernel<false>, SMEM_BYTES);
     if (attr_err == cudaSuccess) attr_err = smem_opt_in<TagPacked>((const void *)kda_chunk_tc_kernel<true>, SMEM_BYTES);
     if (attr_err != cudaSuccess) return attr_err;
+    const WaitHooks hk = wait_hooks();
     TcParams p{(const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.g,
-               (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err, a.cu};
+               (const __nv_bfloat16 *)a.beta, a.s0, (__nv_bfloat16 *)a.out, a.sT, a.T, a.H, a.err, a.cu,
+               hk.wait_ns, hk.skip_load_chunk};
     if (a.cu) kda_chunk_tc_kernel<true><<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
     else kda_chunk_tc_kernel<false><<<a.B * a.H, NT, SMEM_BYTES, s>>>(mq, mk, mv, mg, mo, p);
     return cudaGetLastError();

@@ -82,6 +82,17 @@ bool chunk_f32_supported(const ChunkArgs &a);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 bool chunk_tc_supported(const ChunkArgs &a);
 
+// Limit of every bounded mbarrier wait in the tensor-core kernels, and an injected failure
+// (the tile load of chunk `skip_load_chunk` is never issued; -1: none).  Process-wide, read at
+// each launch; set through kda_set_wait_test_hooks.
+struct WaitHooks {
+    unsigned long long wait_ns;
+    int skip_load_chunk;
+};
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+WaitHooks wait_hooks();
+void set_wait_hooks(unsigned long long wait_ns, int skip_load_chunk);
+
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t s);
 cudaError_t launch_epilogue(const EpilogueArgs &a, cudaStream_t s);

@@ -66,6 +66,17 @@ KDA_DEVICE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *
     }
 }
 
+// Wait on an mbarrier phase for at most `timeout_ns` of wall time, with no abort flag and no
+// error report (used to drain operations already in flight).  Returns false if it gave up.
+KDA_DEVICE bool mbar_wait_timed(uint64_t *bar, uint32_t parity, uint64_t timeout_ns)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > timeout_ns) return false;
+    return true;
+}
+
 // ------------------------------------------------------------------ cp.async (4 bytes)
 // Global -> shared copy of one aligned 32-bit word without a register: src_bytes (0, 2 or 4)
 // are read from src, the rest of the word is zero-filled.  src must be 4-byte aligned.

@@ -62,6 +62,8 @@ def _load():
     lib.kda_layer_decode_step.argtypes = [vp] * 12 + [f] + [vp] * 3 + [f] + [vp] * 2 + [i] * 4 + [i, vp]
     lib.kda_layer_decode_step.restype = i
     lib.kda_check_device_error.argtypes = [vp]
+    lib.kda_set_wait_test_hooks.restype = i
+    lib.kda_set_wait_test_hooks.argtypes = [ctypes.c_ulonglong, i]
     return lib
 
 
@@ -71,7 +73,7 @@ EXPORTED_SYMBOLS = ("kda_status_string", "kda_abi_version", "kda_forward_chunked
                     "kda_decode_step", "kda_layer_workspace_size", "kda_layer_forward",
                     "kda_layer_forward_noalloc", "kda_layer_decode_step", "kda_forward_chunked_varlen",
                     "kda_backward_workspace_size", "kda_backward_chunked", "kda_layer_forward_varlen",
-                    "kda_check_device_error")
+                    "kda_check_device_error", "kda_set_wait_test_hooks")
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 
@@ -387,6 +389,12 @@ def kda_layer_forward_noalloc(q_raw, k_raw, v_raw, conv_q, conv_k, conv_v, g_raw
 def kda_check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel flagged a bounded-wait timeout or CUDA error."""
     _check(_lib.kda_check_device_error(_stream(stream)), "kda_check_device_error")
+
+
+def kda_set_wait_test_hooks(wait_limit_ns=0, skip_load_chunk=-1):
+    """Limit of the tensor-core kernels' bounded waits (0: the default 2 s) and an injected
+    failure (the tile load of chunk `skip_load_chunk` is never issued; -1: off).  Process-wide."""
+    _check(_lib.kda_set_wait_test_hooks(int(wait_limit_ns), int(skip_load_chunk)), "kda_set_wait_test_hooks")
 
 
 # short names

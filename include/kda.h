@@ -22,6 +22,7 @@
  *   kda_layer_decode_step        one decode step of the layer core with a conv cache
  *   kda_backward_chunked         gradients of the recurrence's inputs
  *   kda_*_workspace_size, kda_check_device_error, kda_status_string, kda_abi_version
+ *   kda_set_wait_test_hooks      wait limit and failure injection for the failure path
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless a comment says otherwise; the caller owns
@@ -83,9 +84,11 @@ int kda_abi_version(void);
  *   final_state   [B, H, dk, dv]  fp32, or NULL to skip; may equal initial_state
  *                                 (in-place state passing)
  *   chunk         must be 64.
- * Supported: io KDA_F32 with dk, dv in {64, 128}; io KDA_BF16 with dk = dv = 128
- * (tensor-core path) or dk = dv = 64.  T = 0 is valid: out is untouched and
- * final_state receives initial_state (or zeros).
+ * Supported: dk, dv in {64, 128} in either io dtype.  io KDA_BF16 with dk = dv = 128 runs
+ * on the tcgen05 tensor-core kernel only: on a device or driver where that kernel cannot
+ * run the call returns KDA_ERR_UNSUPPORTED (no slower kernel is substituted).  io KDA_F32
+ * and the other bf16 head-dim pairs run exact fp32 CUDA-core kernels.  T = 0 is valid: out
+ * is untouched and final_state receives initial_state (or zeros).
  */
 kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, const void *g,
                                  const void *beta, const float *initial_state, void *out,
@@ -283,6 +286,24 @@ kda_status_t kda_layer_decode_step(const void *q_raw, const void *k_raw, const v
                                    const void *b_raw, const void *o_gate_raw, const float *o_norm_w,
                                    float norm_eps, float *state, void *out, int B, int H, int dk, int dv,
                                    kda_dtype_t io, kda_stream_t stream);
+
+/*
+ * kda_set_wait_test_hooks — the failure path of the tensor-core kernels, made testable
+ * without a GPU fault.  Those kernels wait on their own mbarriers (tile loads, MMA
+ * completion) with a time limit; a wait that runs out sets the device error word, makes
+ * the whole CTA stop, wait for everything it already issued (loads, MMAs, copies, stores),
+ * free its tensor memory and return, so the context stays usable and the next
+ * kda_check_device_error returns KDA_ERR_TIMEOUT.  The paper has no counterpart to this
+ * entry point.
+ *   wait_limit_ns    limit of each such wait, in ns of %globaltimer; 0 restores the
+ *                    default of 2 s
+ *   skip_load_chunk  >= 0: in every later launch, the tile load of that chunk index is
+ *                    never issued, so the wait for it runs out after the limit (the
+ *                    kernel's outputs from that chunk on are then unspecified); -1: off
+ * The settings are process-wide and read at each launch of those kernels; change them only
+ * while no call is being made from another host thread.  Always returns KDA_OK.
+ */
+kda_status_t kda_set_wait_test_hooks(unsigned long long wait_limit_ns, int skip_load_chunk);
 
 /*
  * Synchronises `stream`, then reports and clears the library's device error word

@@ -52,7 +52,7 @@ def test_status_strings(lib):
         s = lib.kda_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.kda_status_string(99) == b"unknown status"
-    assert lib.kda_abi_version() == 102
+    assert lib.kda_abi_version() == 103
 
 
 P = ctypes.c_void_p
@@ -79,6 +79,17 @@ def test_forward_chunked_rejects_bad_arguments(lib):
     assert _chunked(lib, s0=MIS) == 3
     assert _chunked(lib, sT=MIS) == 3
     assert _chunked(lib, B=1 << 20, T=1 << 20) == 2
+    # beta of the tensor-core shape must be aligned like every other tensor
+    assert _chunked(lib, beta=P(0x100002), dk=128, dv=128, io=1) == 3
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="needs a machine without an sm_100 GPU")
+def test_tensor_core_shape_has_no_slower_substitute(lib):
+    """bf16 at dk = dv = 128 runs on the tcgen05 kernel only: where that kernel cannot run (here:
+    no B200), the call is refused before any launch instead of running another kernel."""
+    assert _chunked(lib, dk=128, dv=128, io=1) == 2
+    assert lib.kda_forward_chunked_varlen(A16, A16, A16, A16, A16, None, A16, None, A16, 2, 100, 2, 128, 128,
+                                          64, 1, None) == 2
 
 
 def test_forward_chunked_varlen_rejects_bad_arguments(lib):
