@@ -432,7 +432,10 @@ def run_ours(args):
             "tokens_per_s": round(ws * Bd / (ms_ld / 1e3), 1),
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
-                         "kernel": "kda_layer_decode", "bytes_per_launch": state_bytes + io_bytes}}
+                         "frac_of_8TBs": round(gbs / 8000.0, 4), "traffic": traffic_for("kda_layer_decode"),
+                         "kernel": "kda_layer_decode", "bytes_per_launch": state_bytes + io_bytes,
+                         "note": "the state is read and written in place (same lines), which a plain "
+                                 "copy's read-A/write-B peak does not model; frac can exceed 1"}}
         launches_per["layer_decode"] = wd["steps"] * reps
         del state, caches, steps_in, od, Ld, fixed
         torch.cuda.empty_cache()
@@ -478,6 +481,10 @@ def run_ours(args):
     cpu = None
     if rank == 0 and ws == 1 and "cpu" not in skip:
         cpu = cpu_baseline_prefill()
+        if "decode" in res:
+            res["decode"]["cpu_baseline"] = cpu_baseline_decode()
+        if "layer" in res:
+            res["layer"]["cpu_baseline"] = cpu_baseline_layer()
 
     gpu_launches = args.steps * (launches_per["prefill"] + launches_per.get("varlen", 0)) + \
         launches_per.get("backward", 0) + launches_per.get("decode", 0) + launches_per.get("layer_decode", 0) + \
@@ -528,6 +535,62 @@ def cpu_baseline_prefill(min_seconds=10.0, max_reps=40):
             "kind": "oracle",
             "sample": f"{reps} runs of {nh} heads x T={w['T']} of the prefill workload (fp64 token "
                       f"recurrence, {token_heads} token-heads, {total:.1f} s); tokens/s = token-heads/s / 96"}
+
+
+def cpu_baseline_decode(min_seconds=3.0, max_reps=20):
+    """The fp64 oracle's decode step on a sample of the decode workload: 4 of the 256
+    sequences, all 96 heads, the 20 chained steps; repeated until about `min_seconds`.
+    Returns the cpu_baseline object in GB/s of the same algorithmic bytes per (b, h) step
+    (state read and written, and the I/O) and in tokens/s."""
+    import oracle
+    from gated_delta_rule_155_b200 import inputs
+
+    w = inputs.WORKLOADS[DECODE]
+    nb = 4
+    dd = inputs.decode_inputs(nb, w["H"], w["dk"], w["dv"], steps=w["steps"], io=w["io"], seed=w["seed"],
+                              s0_std=w["s0_std"])
+    steps = [[x[n].double().numpy() for n in ("q", "k", "v", "g", "beta")] for x in dd["steps"]]
+    cores = oracle.max_threads()
+    reps, total = 0, 0.0
+    while reps < max_reps and (total < min_seconds or reps == 0):
+        st = dd["state"].double().numpy()
+        t0 = time.perf_counter()
+        for x in steps:
+            _, st = oracle.decode(*x, st, nthreads=cores)
+        total += time.perf_counter() - t0
+        reps += 1
+    head_steps = nb * w["H"] * w["steps"] * reps
+    per = 2 * w["dk"] * w["dv"] * 4 + (3 * w["dk"] * 2 + w["dv"] * 2 * 2 + 2)
+    return {"value": round(head_steps * per / total / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "tokens_per_s": round(head_steps / total / w["H"], 1),
+            "sample": f"{reps} runs of {nb} sequences x {w['H']} heads x {w['steps']} chained steps of the decode "
+                      f"workload (fp64 decode step, {total:.1f} s); GB/s of the kernel's algorithmic bytes"}
+
+
+def cpu_baseline_layer(min_seconds=5.0, max_reps=20):
+    """The fp64 layer oracle (conv + SiLU, L2-norm, gate, beta, token recurrence, RMSNorm x
+    sigmoid gate) on the first 8 heads of one T = 16384 sequence of the layer workload;
+    repeated until about `min_seconds`.  tokens/s = token-heads/s / 96."""
+    import oracle
+    from gated_delta_rule_155_b200 import inputs
+
+    w = inputs.WORKLOADS[LAYER]
+    nh, d = 8, w["dk"]
+    L = inputs.layer_inputs(1, w["T"], nh, d, w["dv"], io=w["io"], seed=w["seed"], conv_std=w["conv_std"])
+    arrs = [None if L[n] is None else L[n].double().numpy()
+            for n in ("q_raw", "k_raw", "v_raw", "conv_q", "conv_k", "conv_v", "g_raw", "A_log", "dt_bias",
+                      "b_raw", "o_gate_raw", "o_norm_w")]
+    cores = oracle.max_threads()
+    reps, total = 0, 0.0
+    while reps < max_reps and (total < min_seconds or reps == 0):
+        t0 = time.perf_counter()
+        oracle.layer(*arrs, nthreads=cores)
+        total += time.perf_counter() - t0
+        reps += 1
+    token_heads = nh * w["T"] * reps
+    return {"value": round(token_heads / total / w["H"], 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} runs of {nh} heads x T={w['T']} of the layer workload (fp64 layer core, "
+                      f"{token_heads} token-heads, {total:.1f} s); tokens/s = token-heads/s / {w['H']}"}
 
 
 def run_reference(args):

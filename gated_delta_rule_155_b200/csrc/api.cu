@@ -64,6 +64,10 @@ LayerWorkspace layer_workspace(int B, int T, int H, int dk, int dv)
     return w;
 }
 
+// The layer core runs as one tensor-core kernel (no workspace) for bf16 at dk = dv = 128;
+// other dtypes and head dims run prologue -> exact fp32 chunk kernel -> epilogue.
+bool layer_on_tensor_cores(kda_dtype_t io, int dk, int dv) { return io == KDA_BF16 && dk == 128 && dv == 128; }
+
 // Shapes common to every entry point.
 kda_status_t check_dims(int B, int T, int H, int dk, int dv, kda_dtype_t io)
 {
@@ -110,6 +114,16 @@ kda_status_t layer_core(const void *q_raw, const void *k_raw, const void *v_raw,
     cudaStream_t s = (cudaStream_t)stream;
     if (T == 0) return cuda_status(kda::launch_fill_state(initial_state, final_state,
                                                           (size_t)B * H * dk * dv, s));
+    if (layer_on_tensor_cores(io, dk, dv)) {
+        // one tcgen05 kernel for the whole layer core, no workspace; where it cannot run the call
+        // is refused rather than given to a slower kernel
+        if (((uintptr_t)b_raw & 3) != 0) return KDA_ERR_MISALIGNED;
+        kda::LayerTcArgs la{q_raw, k_raw, v_raw, g_raw, b_raw, o_gate_raw, conv_q, conv_k, conv_v, A_log,
+                            dt_bias, o_norm_w, gate_lower_bound, norm_eps, initial_state, final_state, out,
+                            B, T, H, dk, dv, kda::IO_BF16, error_word(), cu};
+        if (!kda::layer_tc_supported(la)) return KDA_ERR_UNSUPPORTED;
+        return cuda_status(kda::launch_layer_tc(la, s));
+    }
     const int rows = cu ? 1 : B;   // batch rows of the token-major tensors
     const LayerWorkspace w = layer_workspace(rows, T, H, dk, dv);
     if (!workspace || workspace_bytes < w.total) return KDA_ERR_WORKSPACE;
@@ -252,7 +266,7 @@ kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_d
     if (!bytes) return KDA_ERR_INVALID_ARG;
     kda_status_t st = check_dims(B, T, H, dk, dv, io);
     if (st != KDA_OK) return st;
-    *bytes = T == 0 ? 0 : layer_workspace(B, T, H, dk, dv).total;
+    *bytes = (T == 0 || layer_on_tensor_cores(io, dk, dv)) ? 0 : layer_workspace(B, T, H, dk, dv).total;
     return KDA_OK;
 }
 

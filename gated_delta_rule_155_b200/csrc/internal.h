@@ -2,6 +2,7 @@
 // Launchers assume validated arguments; they only configure and launch.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -73,6 +74,23 @@ struct LayerDecodeArgs {
 };
 cudaError_t launch_layer_decode(const LayerDecodeArgs &a, cudaStream_t s);
 
+// The whole layer core (prologue, chunked recurrence, epilogue) in one tcgen05 kernel: bf16
+// I/O, dk = dv = 128, no workspace.
+struct LayerTcArgs {
+    const void *q_raw, *k_raw, *v_raw, *g_raw, *b_raw, *o_gate_raw;   // bf16 [B, T, H, 128] / [B, T, H]
+    const float *conv_q, *conv_k, *conv_v, *A_log, *dt_bias, *gain;
+    float g_lb, eps;
+    const float *s0;
+    float *sT;
+    void *out;
+    int B, T, H, dk, dv;   // packed: B = sequences over a token axis of T rows
+    IoType io;
+    int *err;
+    const int *cu;
+};
+bool layer_tc_supported(const LayerTcArgs &a);
+cudaError_t launch_layer_tc(const LayerTcArgs &a, cudaStream_t s);
+
 // CUDA-core chunked kernel: any supported dtype, dk, dv in {64, 128}.
 cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 // Exact fp32 chunked kernel on CUDA cores for dk = dv = 128 with all-fp32 operands.
@@ -81,6 +99,13 @@ bool chunk_f32_supported(const ChunkArgs &a);
 // tcgen05 chunked kernel: bf16 I/O, dk = dv = 128.
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s);
 bool chunk_tc_supported(const ChunkArgs &a);
+
+// [B, T, H, 128] bf16 -> 4-D TMA map (128, H, T, B) with box (64, 1, box_rows, 1), 128-byte
+// swizzle and zero fill past the extents.  False if the driver entry point is missing.
+bool make_tile_map(CUtensorMap *m, const void *base, int B, int T, int H, int box_rows);
+// The current device is sm_100 (B200); the driver provides cuTensorMapEncodeTiled.
+bool device_is_sm100();
+bool tensor_maps_available();
 
 // Limit of every bounded mbarrier wait in the tensor-core kernels, and an injected failure
 // (the tile load of chunk `skip_load_chunk` is never issued; -1: none).  Process-wide, read at

@@ -90,6 +90,10 @@ def test_tensor_core_shape_has_no_slower_substitute(lib):
     assert _chunked(lib, dk=128, dv=128, io=1) == 2
     assert lib.kda_forward_chunked_varlen(A16, A16, A16, A16, A16, None, A16, None, A16, 2, 100, 2, 128, 128,
                                           64, 1, None) == 2
+    # the layer core's bf16 d = 128 kernel likewise
+    assert lib.kda_layer_forward(A16, A16, A16, A16, A16, A16, A16, A16, None, ctypes.c_float(-5.0), A16, A16,
+                                 None, ctypes.c_float(1e-6), None, A16, None, None, 0, 1, 40, 2, 128, 128, 1,
+                                 None) == 2
 
 
 def test_forward_chunked_varlen_rejects_bad_arguments(lib):
@@ -160,18 +164,21 @@ def test_layer_decode_rejects_bad_arguments(lib):
 
 def test_layer_workspace_and_argument_checks(lib):
     n = ctypes.c_size_t(0)
-    assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, ctypes.byref(n)) == 0
+    # fp32 I/O runs prologue -> fp32 chunk kernel -> epilogue through a workspace
+    assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 0, ctypes.byref(n)) == 0
     N = 2 * 16 * 3
     assert n.value >= 4 * N * (3 * 128 + 128 + 1 + 128)
-    assert lib.kda_layer_workspace_size(2, 0, 3, 128, 128, 1, ctypes.byref(n)) == 0 and n.value == 0
+    # bf16 at d = 128 is one tensor-core kernel and needs none
+    assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, ctypes.byref(n)) == 0 and n.value == 0
+    assert lib.kda_layer_workspace_size(2, 0, 3, 128, 128, 0, ctypes.byref(n)) == 0 and n.value == 0
     assert lib.kda_layer_workspace_size(2, 16, 3, 128, 128, 1, None) == 1
     assert lib.kda_layer_workspace_size(2, 16, 3, 100, 128, 1, ctypes.byref(n)) == 2
 
-    def layer(ws=A16, ws_bytes=1 << 40, q=A16, eps=1e-6, lb=float("-inf"), **kw):
+    def layer(ws=A16, ws_bytes=1 << 40, q=A16, eps=1e-6, lb=float("-inf"), io=0, **kw):
         return lib.kda_layer_forward(q, A16, A16, A16, A16, A16, A16, A16, None, ctypes.c_float(lb),
                                      A16, A16, None,
                                      ctypes.c_float(eps), None, A16, None, ws, ws_bytes,
-                                     kw.get("B", 1), kw.get("T", 16), kw.get("H", 2), 128, 128, 1, None)
+                                     kw.get("B", 1), kw.get("T", 16), kw.get("H", 2), 128, 128, io, None)
     assert layer(q=None) == 1
     assert layer(eps=-1.0) == 1
     assert layer(lb=1.0) == 1

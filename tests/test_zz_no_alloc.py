@@ -62,10 +62,11 @@ def test_noalloc_matches_layer_forward_on_two_calls(kda, io):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(kda):
     lib = kda.library()
-    need = kda.kda_layer_workspace_size(4, 8192, 96, 128, 128, torch.bfloat16)
+    # fp32 I/O runs through the workspace; this size needs far more than the built-in scratch
+    need = kda.kda_layer_workspace_size(4, 8192, 96, 128, 128, torch.float32)
     assert need > kda.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x100000)   # never dereferenced: the call is refused before any launch
     st = lib.kda_layer_forward_noalloc(*([fake] * 8), None, ctypes.c_float(float("-inf")), fake, fake, None,
                                        ctypes.c_float(1e-6),
-                                       None, fake, None, 4, 8192, 96, 128, 128, 1, None)
+                                       None, fake, None, 4, 8192, 96, 128, 128, 0, None)
     assert st == 6  # KDA_ERR_WORKSPACE
