@@ -9,13 +9,13 @@
 //                       K^ = Gamma*K, K~ = exp(G_C - G)*K and the Gram operands (below).
 //   Gram (tcgen05)      [Q;K] rows x CV_I columns -> P (j <= i) and A' (j < i) in one
 //                       M=128, N=160, K=128 MMA, plus a residual MMA for the diagonal blocks.
-//   inverse (CUDA)      T = (I + Diag(beta) A')^{-1} Diag(beta), column-parallel forward
-//                       substitution in fp32 — while the tensor cores compute Y^T = S^T K^^T
-//                       and O^T = S^T Q^^T.
+//   inverse (CUDA)      T = (I + Diag(beta) A')^{-1} Diag(beta), blocked, fp32 — while the
+//                       tensor cores compute O^T = S^T Q^^T and Y^T = S^T K^^T.
 //   U (tcgen05)         U^T = V^T T^T - Y^T T^T, i.e. U = T (V - K^ S).
 //   chain (tcgen05)     O^T += U^T P^T;  S^T <- S^T Diag(exp G_C) + U^T K~.
-// The products that read the state (Y = K^ S and S^T Q^^T) use it split into bf16 hi + lo
-// parts in tensor memory.
+// The product that reads the state for the output (S^T Q^^T) runs as a kind::tf32 MMA with
+// the fp32 state itself as the TMEM A operand; Y = K^ S uses the state split into bf16
+// hi + lo parts.
 //
 // Overflow-safe Gram factorisation.  exp(G_i - G_j) (j <= i) spans far more than the
 // fp32 range over a chunk, so it is never formed as exp(G_i) exp(-G_j).  Row i of
@@ -33,8 +33,8 @@
 // formed exactly in fp32 from the raw inputs, the diagonal 16x16 blocks of the Gram get a
 // second MMA with the rounding residuals (R_lo CVd + R CVd_lo), U, Y, P and K~ enter their
 // products as hi + lo bf16 pairs (O += U_hi P_hi + U_lo P_hi + U_hi P_lo,
-// S += K~_hi^T (U_hi + U_lo) + K~_lo^T U_hi), and so do the state and Q^ in the O init
-// (S_hi Q^_hi + S_lo Q^_hi + S_hi Q^_lo).
+// S += K~_hi^T (U_hi + U_lo) + K~_lo^T U_hi), and the state is read at tf32 precision from
+// its fp32 copy for S^T Q^^T (Q^ kept in fp32).
 #include <cuda.h>
 
 #include <atomic>
@@ -69,21 +69,22 @@ constexpr int GR_R = 0, GR_CV = 32768;                                // inside 
 constexpr int ST_KLO = 65536;
 constexpr int R_CB = 16384;                      // R: 128 rows x 128 B per channel block
 constexpr int CV_ROWS = 160, CV_CB = CV_ROWS * 128;
-// X1 (32 KB): Q^ as bf16 hi (16 KB) + lo (16 KB), K-major [i][c] like the stage tiles, from
-// pass C until the O-init MMA has run; before that (from the next chunk's pass A, which runs
-// during this chunk's last MMAs) each thread keeps its in-half prefix of g in its own Q^ slots
+// X1 (32 KB): Q^ in fp32 (tf32 K-major [i][c]), from prep until the O-init MMA (issued
+// after the Gram readback) has run
 // X2 (32 KB): R_lo (prep -> Gram); then A and L^{-1} in fp32 (inverse)
 // P and P_lo (bf16 K-major [i][j], 8 KB each) take the stage's q tile once the Gram MMAs have
 // read the residual columns kept there; T (bf16 K-major [i][j], 8 KB) sits in the factor
 // table; the O tile is staged in the stage's V tile
 constexpr int OFF_X1 = 2 * REG_BYTES;
-constexpr int OFF_QH = OFF_X1, OFF_QL = OFF_X1 + 16384;   // Q^ hi, lo: 2 channel blocks x 64 rows x 128 B
+constexpr int OFF_QH = OFF_X1;                   // 32 KB: 4 K-blocks of 32 fp32 x 64 rows
 constexpr int ST_P = ST_Q, ST_PL = ST_Q + 8192;  // inside the stage region
 constexpr int OFF_X2 = OFF_X1 + 32768;
-// A transposed, fp32 [64][64] (AT[j][i] = A[i][j]): the Gram readback writes a column segment
-// per thread (consecutive i across lanes) and the forward substitution reads one column of A
-// per step (consecutive rows across lanes), both free of bank conflicts.
-constexpr int OFF_AT = OFF_X2;
+// A and L^{-1}: fp32 [64][AST]; the row stride of 68 floats shifts consecutive rows by four
+// banks, so column reads and row-segment writes spread over all banks.  L^{-1} runs 2 KB past
+// X2 into the factor table, which is dead between prep and the next chunk.
+constexpr int AST = 68;
+constexpr int OFF_A32 = OFF_X2;
+constexpr int OFF_LINV = OFF_X2 + 64 * AST * 4;
 // per-(block, channel) table, fp32 rows of FSTRIDE (128 channels + padding that puts the
 // four blocks of one channel in different banks): fG, fL, fM for blocks 0..3, the half-block
 // log-decays (row FT_HS + 2 B + half: sum of g over tokens 8 half .. 8 half + 7 of block B),
@@ -92,7 +93,7 @@ constexpr int FSTRIDE = 136;
 constexpr int FT_G = 0, FT_L = 4, FT_M = 8, FT_HS = 12, FT_C = 20;   // row numbers
 constexpr int FT_BYTES = 26 * FSTRIDE * 4;
 constexpr int OFF_FT = OFF_X2 + 32768;
-constexpr int OFF_T = OFF_FT + 2048;             // 1024-aligned
+constexpr int OFF_T = OFF_FT + 2048;             // past L^{-1}'s overhang, 1024-aligned
 constexpr int OFF_MISC = OFF_FT + FT_BYTES;
 constexpr int MS_BADMASK = 0;                    // uint32 [4][4]: channels with L_B < BAD_LOG, per block
 constexpr int MS_GC = 64;                        // fp32 [128] chunk decay exp(G_C)
@@ -102,14 +103,14 @@ constexpr int MS_BAR = 1856;                     // uint64 [5]: tma0, tma1, mma,
 constexpr int MS_TSLOT = 1896;                   // uint32
 constexpr int MS_ABORT = 1900;                   // int
 constexpr int MS_DRAIN = 1904;                   // uint64: MMA drain after an abort
-constexpr int MS_BAR_O2 = 1912;                  // uint64: the chunk's O MMAs
 constexpr int MS_BRAW = 1920;                    // uint32 [2][64]: beta words in flight (cp.async)
 constexpr int MISC_BYTES = 2432;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-static_assert(OFF_AT + 64 * 64 * 4 <= OFF_X2 + 32768, "A^T fits in X2");
+static_assert(OFF_LINV + 64 * AST * 4 <= OFF_MISC, "L^{-1} stays clear of the barriers");
 static_assert(OFF_MISC % 16 == 0 && OFF_FT % 16 == 0 && OFF_T % 1024 == 0 && OFF_T + 8192 <= OFF_MISC, "alignment");
 __host__ __device__ constexpr int fc_slot(int B, int I) { return B == 0 ? I - 1 : (B == 1 ? I + 1 : 5); }
+KDA_DEVICE int aidx(int i, int j) { return i * AST + j; }
 
 // tensor memory columns
 constexpr uint32_t TM_S = 0;       // fp32 S^T, 128 cols
@@ -175,8 +176,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
     uint64_t *bar_drain = (uint64_t *)(misc + MS_DRAIN);
-    uint64_t *bar_o2 = (uint64_t *)(misc + MS_BAR_O2);
-    float *AT = (float *)(sm + OFF_AT);
+    float *A32 = (float *)(sm + OFF_A32);
+    float *LINV = (float *)(sm + OFF_LINV);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
@@ -197,8 +198,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(bar_mma, 1);
         mbar_init(bar_o, 1);
         mbar_init(bar_y, 1);
-        mbar_init(bar_drain, 2);   // the two MMA-issuing threads
-        mbar_init(bar_o2, 1);
+        mbar_init(bar_drain, 3);   // the three MMA-issuing threads
         *abort_flag = 0;
         for (int i = 0; i < 16; ++i) badmask[i] = 0u;
         fence_mbar_init();
@@ -256,6 +256,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     constexpr uint32_t id_gram = idesc_bf16(128, CV_ROWS, false, false);
     constexpr uint32_t id_corr = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t id_o0 = idesc_tf32(128, 64, false, false);
     constexpr uint32_t id_wt = idesc_bf16(128, 64, true, false);
     constexpr uint32_t id_opn = idesc_bf16(128, 64, false, false, true);
     constexpr uint32_t id_op = idesc_bf16(128, 64, false, false);
@@ -279,43 +280,41 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     };
     if (tid < CK && nchunks > 0) beta_async(0);
 
-    constexpr float INV_SC = 7.523164e-37f;    // SC = 2^120, INV_SC = 2^-120
-    constexpr float LN_SC = 83.17766f;         // 120 ln 2
-    // Token mapping of passes A and C: warp (pr, cq, th) takes token position pp = lane & 7
-    // of the half th of block pr (s = 0) and of block 3 - pr (s = 1), so every warp carries
-    // the same number of later-block Gram columns; lane >> 3 picks 8 of the 32 channels of
-    // quarter cq.
-    const int pr = warp & 1;
-    const int cq = (warp >> 1) & 3;   // channel quarter (32 channels)
-    const int th = warp >> 3;         // token half of the block
-    const int pp = lane & 7;          // token position inside the half
-    const int a = 4 * (cq & 1) + (lane >> 3);   // 16-byte chunk inside the channel block
-    const int cb = cq >> 1;           // channel block (64 channels)
-    const int c0 = 64 * cb + 8 * a;
-    auto ftab = [&](int row, float (&f)[8]) {
-        const float *src = FT + row * FSTRIDE + c0;
-        const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
-        f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
-    };
-    // ============================================================ prep, passes A and B
-    // For chunk nn: wait for its tiles, take its beta, the in-half prefix of g (pass A) and
-    // the factor table (pass B).  Chunk n + 1's runs while the tensor pipe executes chunk n's
-    // O and state MMAs: it writes only the factor table, beta, the decay exp(G_C) and the
-    // bad-channel masks, all consumed by chunk n before those MMAs were issued, and X1.
-    // Returns false when the wait for the tiles gave up (the same for the whole CTA).
-    auto prep_ab = [&](int nn) -> bool {
-        const int X = nn & 1;
-        const uint8_t *stg = sm + (X ? OFF_REG1 : OFF_REG0);
-        const int t0 = nn * CK;
-        mbar_wait_bounded(&bar_tma[X], (uint32_t)((nn >> 1) & 1), abort_flag, p.err, p.wait_ns);
+    for (int n = 0; n < nchunks; ++n) {
+        const int X = n & 1;
+        uint8_t *stg = sm + (X ? OFF_REG1 : OFF_REG0);
+        uint8_t *gro = sm + (X ? OFF_REG0 : OFF_REG1);
+        const int t0 = n * CK;
+
+        mbar_wait_bounded(&bar_tma[X], (uint32_t)((n >> 1) & 1), abort_flag, p.err, p.wait_ns);
+
+        // ============================================================ prep
         if (tid < CK) {
             cp_async_wait_all();
             const int t = t0 + tid;
-            const uint32_t wv = BRAW[(nn & 1) * CK + tid];
+            const uint32_t wv = BRAW[(n & 1) * CK + tid];
             const bool hi = t < T && (((uintptr_t)(p.beta + (size_t)(row0 + t) * p.H + h)) & 2);
             BETAsm[tid] = __uint_as_float(hi ? (wv & 0xffff0000u) : (wv << 16));
-            if (nn + 1 < nchunks) beta_async(nn + 1);
+            if (n + 1 < nchunks) beta_async(n + 1);
         }
+        constexpr float INV_SC = 7.523164e-37f;    // SC = 2^120, INV_SC = 2^-120
+        constexpr float LN_SC = 83.17766f;         // 120 ln 2
+        // Token mapping of passes A and C: warp (pr, cq, th) takes token position pp = lane & 7
+        // of the half th of block pr (s = 0) and of block 3 - pr (s = 1), so every warp carries
+        // the same number of later-block Gram columns; lane >> 3 picks 8 of the 32 channels of
+        // quarter cq.
+        const int pr = warp & 1;
+        const int cq = (warp >> 1) & 3;   // channel quarter (32 channels)
+        const int th = warp >> 3;         // token half of the block
+        const int pp = lane & 7;          // token position inside the half
+        const int a = 4 * (cq & 1) + (lane >> 3);   // 16-byte chunk inside the channel block
+        const int cb = cq >> 1;           // channel block (64 channels)
+        const int c0 = 64 * cb + 8 * a;
+        auto ftab = [&](int row, float (&f)[8]) {
+            const float *src = FT + row * FSTRIDE + c0;
+            const float4 u0 = *(const float4 *)src, u1 = *(const float4 *)(src + 4);
+            f[0] = u0.x; f[1] = u0.y; f[2] = u0.z; f[3] = u0.w; f[4] = u1.x; f[5] = u1.y; f[6] = u1.z; f[7] = u1.w;
+        };
         // Rows at or past the end of a packed sequence (the next sequence's tokens) enter as
         // g = 0 and k = 0: they then add nothing to the decays, A, P's columns, Y or the state
         // update, and their own output rows are not stored.  (Fixed length: the tensor maps'
@@ -350,14 +349,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 *(float4 *)dst = make_float4(Gh[s][0], Gh[s][1], Gh[s][2], Gh[s][3]);
                 *(float4 *)(dst + 4) = make_float4(Gh[s][4], Gh[s][5], Gh[s][6], Gh[s][7]);
             }
-            // kept until pass C in this thread's own Q^ hi and lo slots (X1 is free from the O
-            // init on)
-            *(float4 *)(sm + OFF_QH + cb * 8192 + swz(i, a)) = make_float4(Gh[s][0], Gh[s][1], Gh[s][2], Gh[s][3]);
-            *(float4 *)(sm + OFF_QL + cb * 8192 + swz(i, a)) = make_float4(Gh[s][4], Gh[s][5], Gh[s][6], Gh[s][7]);
         }
         __syncthreads();
-        if (*abort_flag) return false;   // the wait for this chunk's tiles gave up
-        tma_consumed = nn + 1;
+        if (*abort_flag) break;   // the wait for this chunk's tiles gave up
+        tma_consumed = n + 1;
         // pass B, one (block, channel) per thread: block log-decays L_J and the factors
         //   fG = exp(G_blockstart)      fL = exp(G_C - G_blockend)
         //   fM = exp(-L_B / 2) / SC     (block-start reference, 1 / SC, where L_B < BAD_LOG)
@@ -393,26 +388,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             if (Bq == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
         }
-        // the previous chunk's O stores must have read their tile before this chunk's pass C
-        // writes Gram operands over it
+        // the previous chunk's O tile (its stage region takes this chunk's Gram operands in pass
+        // C) must have been read out by its TMA store
         if (tid == 0) bulk_wait_read_all();
         __syncthreads();
-        return true;
-    };
-
-    bool alive = nchunks > 0 && prep_ab(0);
-    for (int n = 0; alive && n < nchunks; ++n) {
-        const int X = n & 1;
-        uint8_t *stg = sm + (X ? OFF_REG1 : OFF_REG0);
-        uint8_t *gro = sm + (X ? OFF_REG0 : OFF_REG1);
-        const int t0 = n * CK;
-
-        // Rows at or past the end of a packed sequence (the next sequence's tokens) enter as
-        // g = 0 and k = 0: they then add nothing to the decays, A, P's columns, Y or the state
-        // update, and their own output rows are not stored.  (Fixed length: the tensor maps'
-        // zero fill past T does the same.)
-        const int nvalid = T - t0;
-        const bool tail = PACKED && nvalid < CK;   // the same for the whole block
         // pass C, per token.  With SC = 2^120:
         //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
         //   E2 = SC exp(G_blockend - G_i)    (excludes token i)
@@ -427,17 +406,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t off = cb * 8192 + swz(i, a);
                 float Gin[8], Lb[8];
                 {
-                    // G_i - G_blockstart = in-half prefix (pass A, from the Q^ slots) + the first
-                    // half's sum; L_B
+                    // G_i - G_blockstart = in-half prefix (+ the first half's sum); L_B
                     float h0[8], h1[8];
                     ftab(FT_HS + 2 * B, h0);
                     ftab(FT_HS + 2 * B + 1, h1);
-                    const float4 g0 = *(const float4 *)(sm + OFF_QH + off);
-                    const float4 g1 = *(const float4 *)(sm + OFF_QL + off);
-                    const float gh[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        Gin[e] = gh[e] + (th ? h0[e] : 0.0f);
+                        Gin[e] = Gh[s][e] + (th ? h0[e] : 0.0f);
                         Lb[e] = h0[e] + h1[e];
                     }
                 }
@@ -462,7 +437,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     E1[e] = __expf(Gin[e] + LN_SC);
                     E2[e] = __expf(Lb[e] - Gin[e] + LN_SC);
                 }
-                // Q^ = Gamma q as bf16 hi + lo (K-major, like the stage tiles), Gamma_i = (E1 / SC) fG
+                // Q^ = Gamma q (fp32 K-major tile for the tf32 MMA), Gamma_i = (E1 / SC) fG
                 ftab(FT_G + B, f);
                 float gam[8];
 #pragma unroll
@@ -471,13 +446,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     o[e] = qf[e] * gam[e];
                 }
                 {
-                    const uint4 hq = pack8(o);
-                    float hf[8], lo[8];
-                    unpack8(hq, hf);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) lo[e] = o[e] - hf[e];
-                    *(uint4 *)(sm + OFF_QH + off) = hq;
-                    *(uint4 *)(sm + OFF_QL + off) = pack8(lo);
+                    uint8_t *qh = sm + OFF_QH + (2 * cb + (a >> 2)) * 8192;
+                    *(float4 *)(qh + swz(i, 2 * (a & 3))) = make_float4(o[0], o[1], o[2], o[3]);
+                    *(float4 *)(qh + swz(i, 2 * (a & 3) + 1)) = make_float4(o[4], o[5], o[6], o[7]);
                 }
                 // K^ = Gamma k (in place)
 #pragma unroll
@@ -556,26 +527,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (*abort_flag) break;   // the previous chunk's state wait gave up
 
         // ============================================================ Gram (MMA)
         if (tid == 0) {
             tc_fence_after();
-            // three independent accumulators, interleaved: a chain of MMAs into one accumulator
-            // waits for each accumulation, so alternating chains keeps the tensor pipe busy.
-            // TM_G: R CV (160 columns); the diagonal-block residuals R_lo CVd into TM_CORR and
-            // R CVd_lo (CVd_lo over the q tile) into TM_O, which the readback adds
             const uint32_t sR = smem_u32(gro + GR_R), sCV = smem_u32(gro + GR_CV);
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + TM_G, sdesc(sR + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
+                       sdesc(sCV + (kk >> 2) * CV_CB + (kk & 3) * 32, 16, 1024), id_gram, kk > 0);
+            // diagonal-block residual: R_lo x CVd (CV rows 0..63) + R x CVd_lo (over the q tile)
             const uint32_t sRL = smem_u32(sm + OFF_X2), sCVL = smem_u32(stg + ST_Q);
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t orr = (kk >> 2) * R_CB + (kk & 3) * 32;
-                mma_ss(tmem + TM_G, sdesc(sR + orr, 16, 1024), sdesc(sCV + (kk >> 2) * CV_CB + (kk & 3) * 32, 16, 1024),
-                       id_gram, kk > 0);
-                mma_ss(tmem + TM_CORR, sdesc(sRL + orr, 16, 1024),
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + TM_CORR, sdesc(sRL + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
                        sdesc(sCV + (kk >> 2) * CV_CB + (kk & 3) * 32, 16, 1024), id_corr, kk > 0);
-                mma_ss(tmem + TM_O, sdesc(sR + orr, 16, 1024), sdesc(sCVL + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                       id_corr, kk > 0);
-            }
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + TM_CORR, sdesc(sR + (kk >> 2) * R_CB + (kk & 3) * 32, 16, 1024),
+                       sdesc(sCVL + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_corr, 1);
             mma_commit(bar_mma);
         }
         mma_wait();
@@ -629,11 +596,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     *(uint4 *)(stg + ST_P + swz(i, j0 >> 3)) = hi;
                     *(uint4 *)(stg + ST_PL + swz(i, j0 >> 3)) = pack8(lo);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) AT[(j0 + e) * 64 + i] = vals[e];
+                    *(float4 *)(A32 + aidx(i, j0)) = make_float4(vals[0], vals[1], vals[2], vals[3]);
+                    *(float4 *)(A32 + aidx(i, j0 + 4)) = make_float4(vals[4], vals[5], vals[6], vals[7]);
                 }
             };
-            uint32_t r[2][8], c8[2][8], d8[2][8];
+            uint32_t r[2][8], c8[2][8];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int m = cg + 4 * u;
@@ -642,7 +609,6 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 } else if (m < nch) {
                     tmem_ld8(tmem + lane_q + TM_G + 8 * m, r[u]);               // own (diagonal) block
                     tmem_ld8(tmem + lane_q + TM_CORR + 8 * m, c8[u]);
-                    tmem_ld8(tmem + lane_q + TM_O + 8 * m, d8[u]);
                 }
             }
             tmem_wait_ld();
@@ -653,8 +619,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     if (m >= 2 * I) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            r[u][e] = __float_as_uint(__uint_as_float(r[u][e]) +
-                                                      (__uint_as_float(c8[u][e]) + __uint_as_float(d8[u][e])));
+                            r[u][e] = __float_as_uint(__uint_as_float(r[u][e]) + __uint_as_float(c8[u][e]));
                     }
                     emit(8 * m, r[u]);
                 } else if (is_q) {
@@ -685,7 +650,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 *ph = vh;
                                 *pl = __float2bfloat16_rn(v - __bfloat162float(vh));
                             } else {
-                                AT[j * 64 + i] += bi * d;
+                                A32[aidx(i, j)] += bi * d;
                             }
                         }
                         w *= __expf(valid ? __bfloat162float(p.g[rowj]) : 0.0f);
@@ -697,69 +662,127 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (*abort_flag) break;   // the Gram wait gave up
         if (tid < 16) badmask[tid] = 0u;   // masks consumed
         // ============================================================ T (warps 0..7) || Y = K^ S (warps 8..15)
-        // Warps 0..7 invert L = I + A and form T.  Warps 8..15 (named barrier 2) split the
-        // chunk-start state S^T into bf16 hi + lo in tensor memory, issue Y^T = S^T K^^T (one
-        // bf16 MMA chain per part, fp32 accumulate), split Y^T the same way and, once the O init
-        // has read the state, decay it by exp(G_C).  After both:
-        // U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T, i.e. U = T (V - K^ S) = U~ - W S, with S
-        // entering at about 2^-16 relative precision.
+        // Warps 0..7 invert L = I + A and form T (named barrier 1).  Warps 8..15 (named barrier
+        // 2) issue the O init, split the chunk-start state S^T into bf16 hi + lo in tensor
+        // memory, issue Y^T = S^T K^^T (one bf16 MMA chain per part, fp32 accumulate), split
+        // Y^T the same way and decay the state by exp(G_C).  After both:  U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T, i.e.
+        // U = T (V - K^ S) = U~ - W S, with S entering at about 2^-16 relative precision.
         if (warp < 8) {
-            // T = (I + A)^{-1} Diag(beta) by forward substitution, column-parallel and free of
-            // barriers: warp w owns 8 columns of L^{-1} = (I + A)^{-1}, four below 32 and four
-            // above, and lane l holds rows l and l + 32 of each.  Step m
-            // broadcasts x_m of each column from its owner lane and updates the rows below m:
-            // x_r -= A[r][m] x_m.  All fp32.
-            int colv[8];   // w < 15 - w < 16 + w < 31 - w < 32 + w < 47 - w < 48 + w < 63 - w
+            // L = I + A, inverted in two levels of 2x2 blocks.  16x16 diagonal inverses
+            // L_II^{-1} by right-looking forward substitution (one column per thread); then each
+            // 32x32 half  [[L_a, 0], [A_ba, L_b]]^{-1} = [[L_a^{-1}, 0], [-L_b^{-1} A_ba L_a^{-1}, L_b^{-1}]]
+            // and the same rule once more for the 64x64 matrix with 32x32 blocks.  Every product
+            // is a full-precision fp32 dot product (16x16 blocks: one output per thread and
+            // half; 32x32 blocks: 4 rows x 1 column per thread).  Scratch (P, Q) lives in A's
+            // unused upper-right 32x32 block.
+            if (tid < 64) {
+                const int Ib = tid >> 4, col = tid & 15;
+                float x[16];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) colv[q] = 16 * (q >> 1) + ((q & 1) ? 15 - warp : warp);
-            float x0[8], x1[8];
+                for (int r = 0; r < 16; ++r) x[r] = r == col ? 1.0f : 0.0f;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                x0[q] = lane == colv[q] ? 1.0f : 0.0f;
-                x1[q] = lane + 32 == colv[q] ? 1.0f : 0.0f;
+                for (int m = 0; m < 15; ++m)
+#pragma unroll
+                    for (int r = m + 1; r < 16; ++r) x[r] -= A32[aidx(16 * Ib + r, 16 * Ib + m)] * x[m];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) LINV[aidx(16 * Ib + r, 16 * Ib + col)] = x[r];
             }
-            // Steps 0..31 change only the four columns below 32 (the others are still zero in
-            // rows 0..31); a step m < colv[q] leaves column q unchanged (its x_m is zero).  The
-            // loop bounds are compile-time constants, so the column chains of a step overlap.
-#pragma unroll 4
-            for (int m = 0; m < 32; ++m) {
-                const float a0 = AT[m * 64 + lane], a1 = AT[m * 64 + 32 + lane];
+            named_bar_sync(1, 256);
+            // dot16(X, xr, xc, Y, yr, yc): sum_m X[xr][xc + m] Y[yr + m][yc], m < 16
+            auto dot16 = [&](const float *Xm, int xr, int xc, const float *Ym, int yr, int yc) -> float {
+                float s0 = 0.0f, s1 = 0.0f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float xm = __shfl_sync(0xffffffffu, x0[q], m);
-                    x0[q] = lane > m ? x0[q] - a0 * xm : x0[q];
-                    x1[q] -= a1 * xm;
+                for (int m4 = 0; m4 < 16; m4 += 4) {
+                    const float4 xv = *(const float4 *)(Xm + aidx(xr, xc + m4));
+                    s0 += xv.x * Ym[aidx(yr + m4 + 0, yc)] + xv.z * Ym[aidx(yr + m4 + 2, yc)];
+                    s1 += xv.y * Ym[aidx(yr + m4 + 1, yc)] + xv.w * Ym[aidx(yr + m4 + 3, yc)];
                 }
-            }
-#pragma unroll 4
-            for (int m = 32; m < 63; ++m) {
-                const float a1 = AT[m * 64 + 32 + lane];
+                return s0 + s1;
+            };
+            {
+                // halves h = 0 (blocks 0, 1) and h = 1 (blocks 2, 3):
+                // P_h = A_{2h+1,2h} L_{2h}^{-1}  ->  scratch rows 0..15, columns 32 + 16 h ..
+                const int r = tid >> 4, c = tid & 15;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float xm = __shfl_sync(0xffffffffu, x1[q], m - 32);
-                    x1[q] = lane + 32 > m ? x1[q] - a1 * xm : x1[q];
+                for (int hh = 0; hh < 2; ++hh)
+                    A32[aidx(r, 32 + 16 * hh + c)] = dot16(A32, 32 * hh + 16 + r, 32 * hh, LINV, 32 * hh, 32 * hh + c);
+                named_bar_sync(1, 256);
+                // T_{2h+1,2h} = -L_{2h+1}^{-1} P_h; the (2h, 2h+1) block is zero
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int ra = 32 * hh, rb = ra + 16;
+                    LINV[aidx(rb + r, ra + c)] = -dot16(LINV, rb + r, rb, A32, 0, 32 + 16 * hh + c);
+                    LINV[aidx(ra + r, rb + c)] = 0.0f;
                 }
+                named_bar_sync(1, 256);
             }
-            // T = L^{-1} Diag(beta) in bf16, K-major [i][j]; its upper part is the zeros above
-            // each column's diagonal
+            {
+                // Q = A_{[2,3],[0,1]} L_{[0,1]}^{-1}: 4 rows x 1 column per thread
+                const int c = tid & 31, rg = tid >> 5;   // rows 4 rg .. 4 rg + 3 of 32
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int j = colv[q];
-                const float bj = BETAsm[j];
-                *(__nv_bfloat16 *)(sm + OFF_T + swz(lane, j >> 3) + 2 * (j & 7)) = __float2bfloat16_rn(x0[q] * bj);
-                *(__nv_bfloat16 *)(sm + OFF_T + swz(lane + 32, j >> 3) + 2 * (j & 7)) = __float2bfloat16_rn(x1[q] * bj);
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    float y[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) y[t] = LINV[aidx(m4 + t, c)];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 xv = *(const float4 *)(A32 + aidx(32 + 4 * rg + q, m4));
+                        acc[q] += xv.x * y[0] + xv.y * y[1] + xv.z * y[2] + xv.w * y[3];
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) A32[aidx(4 * rg + q, 32 + c)] = acc[q];
+                named_bar_sync(1, 256);
+                // T_{[2,3],[0,1]} = -L_{[2,3]}^{-1} Q
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[q] = 0.0f;
+#pragma unroll
+                for (int m4 = 0; m4 < 32; m4 += 4) {
+                    float y[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) y[t] = A32[aidx(m4 + t, 32 + c)];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 xv = *(const float4 *)(LINV + aidx(32 + 4 * rg + q, 32 + m4));
+                        acc[q] += xv.x * y[0] + xv.y * y[1] + xv.z * y[2] + xv.w * y[3];
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) LINV[aidx(32 + 4 * rg + q, c)] = -acc[q];
+                named_bar_sync(1, 256);
+            }
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                // T = L^{-1} Diag(beta), lower triangle, bf16 K-major [i][j]
+                const int idx = tid + 256 * it, i = idx >> 3, jc = idx & 7;
+                const float4 l0 = *(const float4 *)(LINV + aidx(i, 8 * jc)), l1 = *(const float4 *)(LINV + aidx(i, 8 * jc + 4));
+                const float4 b0 = *(const float4 *)(BETAsm + 8 * jc), b1 = *(const float4 *)(BETAsm + 8 * jc + 4);
+                const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                float vals[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) vals[e] = 8 * jc + e <= i ? lv[e] * bv[e] : 0.0f;
+                *(uint4 *)(sm + OFF_T + swz(i, jc)) = pack8(vals);
             }
             fence_proxy_async();
         } else {
             const int hb = (warp - 8) >> 2;   // column half of the TMEM tiles this warp splits
-            // S^T (fp32, key channels 64 hb .. 64 hb + 63) -> bf16 hi + lo, two per column; the
-            // copies are all that the Y and O-init MMAs read, so the state is decayed by exp(G_C)
-            // in the same pass
+            if (tid == NT - 32) {
+                // O^T = S^T Q^^T at tf32 (A = fp32 state in TMEM, 8 key channels per MMA); it
+                // completes on bar_o before the state is decayed
+                tc_fence_after();
+                const uint32_t sQ = smem_u32(sm + OFF_QH);
+                for (int kk = 0; kk < 16; ++kk)
+                    mma_ts_tf32(tmem + TM_O, tmem + TM_S + kk * 8, sdesc(sQ + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                id_o0, kk > 0);
+                mma_commit(bar_o);
+            }
+            // S^T (fp32, key channels 64 hb .. 64 hb + 63) -> bf16 hi + lo, two per column
 #pragma unroll
             for (int cc = 0; cc < 64; cc += 32) {
                 uint32_t r[32], hi[16], lo[16];
-                const uint32_t ta = tmem + lane_q + TM_S + 64 * hb + cc;
-                tmem_ld32(ta, r);
+                tmem_ld32(tmem + lane_q + TM_S + 64 * hb + cc, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -770,29 +793,21 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 tmem_st16(tmem + lane_q + TM_SH + 32 * hb + cc / 2, hi);
                 tmem_st16(tmem + lane_q + TM_SL + 32 * hb + cc / 2, lo);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * GCsm[64 * hb + cc + e]);
-                tmem_st32(ta, r);
             }
             tmem_wait_st();
             tc_fence_before();
             named_bar_sync(2, 256);
             if (tid == 256) {
-                // Y^T = S_hi^T K^^T + S_lo^T K^^T  (K^ = Gamma k, bf16 K-major in the stage), then
-                // O^T = S^T Q^^T as S_hi Q^_hi + S_lo Q^_hi + S_hi Q^_lo (Q^ hi, lo in X1)
+                // Y^T = S_hi^T K^^T + S_lo^T K^^T  (K^ = Gamma k, bf16 K-major in the stage)
                 tc_fence_after();
-                const uint32_t sK = smem_u32(stg + ST_K), sQH = smem_u32(sm + OFF_QH), sQL = smem_u32(sm + OFF_QL);
-                // the Y and O chains alternate (independent accumulators)
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_ts(tmem + TM_Y, tmem + TM_SH + kk * 8, sdesc(sK + o, 16, 1024), id_op, kk > 0);
-                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQH + o, 16, 1024), id_op, kk > 0);
-                    mma_ts(tmem + TM_Y, tmem + TM_SL + kk * 8, sdesc(sK + o, 16, 1024), id_op, 1);
-                    mma_ts(tmem + TM_O, tmem + TM_SL + kk * 8, sdesc(sQH + o, 16, 1024), id_op, 1);
-                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQL + o, 16, 1024), id_op, 1);
-                }
+                const uint32_t sK = smem_u32(stg + ST_K);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + TM_Y, tmem + TM_SH + kk * 8, sdesc(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                           id_op, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + TM_Y, tmem + TM_SL + kk * 8, sdesc(sK + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                           id_op, 1);
                 mma_commit(bar_y);
-                mma_commit(bar_o);
             }
             if (mbar_wait_bounded(bar_y, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns)) {
                 tc_fence_after();
@@ -811,8 +826,22 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tmem_st16(tmem + lane_q + TM_LO32 + 16 * hb, lo);
                 tmem_wait_st();
             }
-            // the O init has read X1 and written TM_O before the section ends
-            mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns);
+            // S^T <- S^T Diag(exp G_C): every reader of the chunk-start state is done once the
+            // O init has completed (the split above and the Y MMAs read the copies)
+            if (mbar_wait_bounded(bar_o, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns)) {
+                tc_fence_after();
+#pragma unroll
+                for (int cc = 0; cc < 64; cc += 32) {
+                    uint32_t sr[32];
+                    const uint32_t ta = tmem + lane_q + TM_S + 64 * hb + cc;
+                    tmem_ld32(ta, sr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sr[e] = __float_as_uint(__uint_as_float(sr[e]) * GCsm[64 * hb + cc + e]);
+                    tmem_st32(ta, sr);
+                }
+                tmem_wait_st();
+            }
         }
         tc_fence_before();
         __syncthreads();
@@ -821,28 +850,25 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ============================================================ U^T = V^T T^T - Y_hi^T T^T - Y_lo^T T^T
         if (tid == 0) {
             tc_fence_after();
-            // two accumulators, interleaved: V T - Y_hi T into TM_U, -Y_lo T into TM_Y (free since
-            // the Y split); the U split adds them
             const uint32_t sV = smem_u32(stg + ST_V), sT_ = smem_u32(sm + OFF_T);
-            for (int kk = 0; kk < 4; ++kk) {
+            for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tmem + TM_U, sdesc(sV + kk * 2048, 8192, 1024), sdesc(sT_ + kk * 32, 16, 1024), id_wt, kk > 0);
-                mma_ts(tmem + TM_Y, tmem + TM_LO32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
                 mma_ts(tmem + TM_U, tmem + TM_HI32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, 1);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ts(tmem + TM_U, tmem + TM_LO32 + kk * 8, sdesc(sT_ + kk * 32, 16, 1024), id_opn, 1);
             mma_commit(bar_mma);
         }
         mma_wait();
         tc_fence_after();
         {
             // U^T fp32 -> bf16 hi and lo A operands (two bf16 per 32-bit column; Y's are consumed)
-            uint32_t r[16], r2[16], r8[8], l8[8];
+            uint32_t r[16], r8[8], l8[8];
             tmem_ld16(tmem + lane_q + TM_U + 16 * cg, r);
-            tmem_ld16(tmem + lane_q + TM_Y + 16 * cg, r2);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float x0 = __uint_as_float(r[2 * e]) + __uint_as_float(r2[2 * e]);
-                const float x1 = __uint_as_float(r[2 * e + 1]) + __uint_as_float(r2[2 * e + 1]);
+                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
                 r8[e] = pack_bf16x2(x0, x1);
                 const float2 hv = unpack_bf16x2(r8[e]);
                 l8[e] = pack_bf16x2(x0 - hv.x, x1 - hv.y);
@@ -858,33 +884,27 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             const uint32_t sP = smem_u32(stg + ST_P), sPL = smem_u32(stg + ST_PL), sG = smem_u32(stg + ST_G);
             const uint32_t sKL0 = smem_u32(sm + OFF_REG0 + ST_KLO), sKL1 = smem_u32(sm + OFF_REG1 + ST_KLO);
-            // the O chain alternates with the state update's main terms; bar_o2 then covers both,
-            // and the K~ lo terms follow on bar_mma
             for (int kk = 0; kk < 4; ++kk) {
                 mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
-                mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
                 mma_ts(tmem + TM_O, tmem + TM_LO32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
-                mma_ts(tmem + TM_S, tmem + TM_LO32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
                 mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sPL + kk * 32, 16, 1024), id_op, 1);
             }
-            mma_commit(bar_o2);
             for (int kk = 0; kk < 4; ++kk) {
+                mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
+                mma_ts(tmem + TM_S, tmem + TM_LO32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
                 // K~ lo, one 64-channel block (state columns) per MMA
                 mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sKL0 + kk * 2048, 8192, 1024), id_s64, 1);
                 mma_ts(tmem + TM_S + 64, tmem + TM_HI32 + kk * 8, sdesc(sKL1 + kk * 2048, 8192, 1024), id_s64, 1);
             }
             mma_commit(bar_mma);
         }
-        // The O MMAs complete on bar_o2 (with the state update's main terms), the K~ lo terms on
-        // bar_mma: O is staged and stored while they run, and so do the next chunk's passes A, B.
-        mbar_wait_bounded(bar_o2, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns);
+        mma_wait();
         tc_fence_after();
         {
             // O^T -> bf16 tile in the stage's V tile (dead since the U~ MMA; the load tiles'
             // layout: 2 channel blocks of [64 rows x 128 B], 128-byte swizzle), then two TMA
-            // stores; rows past T are clipped by the tensor map.  This region takes the next
-            // chunk's Gram operands, so thread 0 waits for the stores' shared-memory reads before
-            // the last barrier of the next chunk's pass B.
+            // stores; rows past T are clipped by the tensor map.  The stores are waited for
+            // (read side) only before the next TMA load into this stage region.
             const int v = 32 * lq + lane;
             uint32_t r[16];
             tmem_ld16(tmem + lane_q + TM_O + 16 * cg, r);
@@ -897,7 +917,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (*abort_flag) break;   // the O wait gave up
+        if (*abort_flag) break;   // the O / state wait gave up
         if (tail) {
             // the last chunk of a packed sequence: its tile's later rows are the next
             // sequence's, so only the valid rows are written, 16 bytes per thread and pass
@@ -912,16 +932,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tma_store_4d(&tm_o, stg + ST_V + 8192, 64, h, tt0 + t0, tb);
             bulk_commit();
         }
-        // the next chunk's passes A and B run while the tensor pipe executes the state MMAs
-        if (n + 1 < nchunks && !prep_ab(n + 1)) break;
-        mma_wait();   // checked after the next barrier, before the next chunk's Gram issue
-        tc_fence_after();
     }
 
     // ---------------------------------------------------------------- final state
-    tc_fence_before();
-    __syncthreads();   // the last state wait's outcome is read by every thread alike
-    tc_fence_after();
     if (p.sT && !*abort_flag) {
         tc_fence_after();
         const int v = 32 * lq + lane;
@@ -935,12 +948,12 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (*abort_flag) {
         // A bounded wait gave up (the flag is read after a block barrier, so the whole CTA is
         // here).  Everything asynchronous this CTA started finishes before its shared and tensor
-        // memory are released: the MMAs of the two issuing threads (one commit each on
+        // memory are released: the MMAs of the three issuing threads (one commit each on
         // bar_drain), a tile load issued but not yet waited for, the beta copies and the bulk
         // stores.  These operations were really issued, so they complete; the waits are
         // bounded all the same.
         constexpr unsigned long long DRAIN_NS = 2000000000ull;
-        if (tid == 0 || tid == 256) mma_commit(bar_drain);
+        if (tid == 0 || tid == 256 || tid == NT - 32) mma_commit(bar_drain);
         if (tid == 0) {
             if (tma_issued > tma_consumed) {
                 const int c = tma_consumed;

@@ -16,8 +16,8 @@
 //                        V, and the Gram operands (the overflow-safe midpoint factorisation of
 //                        the tensor-core prefill, chunk_tc.cu)
 //   Gram (tcgen05)       P (j <= i) and A (j < i) in one M = 128, N = 48, K = 128 MMA group
-//   inverse || Y, O init T = (I + A)^{-1} Diag(beta) by column-parallel forward substitution,
-//                        while the tensor cores compute Y^T = S^T K^^T and O^T = S^T Q^^T
+//   inverse || Y, O init T = (I + A)^{-1} Diag(beta), one column per lane in registers, while
+//                        the tensor cores compute Y^T = S^T K^^T and O^T = S^T Q^^T
 //   U, O, S (tcgen05)    U = T (V - Y);  O += P U;  S <- Diag(exp G_C) S + K~^T U
 //   epilogue             out = gain * cast_bf16(o * rsqrt(mean_v(o^2) + eps)) * sigmoid(z)
 //                        (atlas.klimoza.dev "Kimi-K3 > KDA layers", KimiRMSNorm excerpt;
@@ -63,12 +63,12 @@ constexpr int OFF_STG0 = 0, OFF_STG1 = STAGE;
 // M = 128 MMA also reads the 64 rows after each channel block (other operands; the tensor-memory
 // lanes they produce are never read); columns CV (48 rows: tokens 0..31 with their own block's
 // reference, then block 0's tokens with block 1's), hi and lo.  After the Gram: P hi, lo and T
-// hi, lo ([32 rows][128 B], K-major, columns 0..31 used) and A transposed (fp32 [32][32]).
+// hi, lo ([32 rows][128 B], K-major, columns 0..31 used) and A (fp32 [32][AST], row-major).
 constexpr int OFF_GR = 2 * STAGE;
 constexpr int R_CB = 8192, CV_CB = 6144;
 constexpr int GR_RH = 0, GR_RL = 16384, GR_CVH = 32768, GR_CVL = 32768 + 2 * CV_CB;
 constexpr int GR_BYTES = GR_CVL + 2 * CV_CB;
-constexpr int GR_PH = 0, GR_PL = 4096, GR_TH = 8192, GR_TL = 12288, GR_AT = 16384;
+constexpr int GR_PH = 0, GR_PL = 4096, GR_TH = 8192, GR_TL = 12288, GR_A = 16384, AST = 36;
 // operand tiles ([32 rows][128 channels] bf16, the tile layout)
 constexpr int OFF_QH = OFF_GR + GR_BYTES, OFF_QL = OFF_QH + TILE;   // Q^ hi, lo (K-major B of the O init)
 constexpr int OFF_KH = OFF_QL + TILE;                               // K^ (K-major B of Y)
@@ -97,7 +97,7 @@ constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 static_assert(OFF_GR % 1024 == 0 && OFF_QH % 1024 == 0 && OFF_VL % 1024 == 0 && GR_CVL % 1024 == 0 &&
               (GR_CVH + CV_CB) % 1024 == 0, "operand tiles are 1024-aligned");
-static_assert(GR_AT + 32 * 32 * 4 <= GR_BYTES && OFF_MISC % 16 == 0, "layout");
+static_assert(GR_A + 32 * AST * 4 <= GR_BYTES && OFF_MISC % 16 == 0, "layout");
 
 // tensor memory columns
 constexpr uint32_t TM_S = 0;     // fp32 S^T, 128
@@ -134,6 +134,14 @@ KDA_DEVICE uint4 pack8(const float (&f)[8])
     return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                       pack_bf16x2(f[6], f[7]));
 }
+// Activations with the fast reciprocal and logarithm (relative errors about 2^-21, well below
+// the 2^-16 the chunk algebra keeps): the IEEE division and log1pf cost several times more.
+KDA_DEVICE float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+KDA_DEVICE float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+// log(1 + e^x) = max(x, 0) + log(1 + e^-|x|); 1 + e^-|x| lies in (1, 2], where the logarithm
+// keeps its relative accuracy
+KDA_DEVICE float softplus_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))); }
+
 // x -> bf16 hi and the bf16 residual lo
 KDA_DEVICE void split8(const float (&x)[8], uint4 &hi, uint4 &lo)
 {
@@ -175,7 +183,7 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *bar_drain = bar_tma + 6;
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
-    float *AT = (float *)(gr + GR_AT);
+    float *A32 = (float *)(gr + GR_A);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
@@ -305,31 +313,33 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int t = t0 + tid;
             const uint32_t wv = BRAW[(nn & 1) * CK + tid];
             const bool hi = t < T && (((uintptr_t)(p.b + (size_t)(row0 + t) * p.H + h)) & 2);
-            BETAsm[tid] = sigmoidf_(__uint_as_float(hi ? (wv & 0xffff0000u) : (wv << 16)));
+            BETAsm[tid] = sigmoid_fast(__uint_as_float(hi ? (wv & 0xffff0000u) : (wv << 16)));
             if (nn + 1 < nchunks) b_async(nn + 1);
         }
         const int nvalid = T - t0;
         // short conv + SiLU: y[c] = SiLU(sum_u w[c][u] x[i - 3 + u][c]); rows before the chunk
         // come from the previous chunk's tile, or are zero at the sequence start
         auto conv = [&](int st_off, int tensor, float (&y)[8]) {
-            float acc[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+            float x[4][8];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int r = ti - 3 + u;
-                float x[8];
-                if (r >= 0) unpack8(*(const uint4 *)(stg + st_off + cb * CBT + swz(r, ca)), x);
-                else if (nn > 0) unpack8(*(const uint4 *)(prv + st_off + cb * CBT + swz(r + CK, ca)), x);
+                if (r >= 0) unpack8(*(const uint4 *)(stg + st_off + cb * CBT + swz(r, ca)), x[u]);
+                else if (nn > 0) unpack8(*(const uint4 *)(prv + st_off + cb * CBT + swz(r + CK, ca)), x[u]);
                 else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+                    for (int e = 0; e < 8; ++e) x[u][e] = 0.0f;
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] += CW[(tensor * DD + c0 + e) * 4 + u] * x[e];
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = siluf_(acc[e]);
+            for (int e = 0; e < 8; ++e) {
+                const float4 w = *(const float4 *)(CW + (tensor * DD + c0 + e) * 4);
+                float acc = w.x * x[0][e];
+                acc = fmaf(w.y, x[1][e], acc);
+                acc = fmaf(w.z, x[2][e], acc);
+                acc = fmaf(w.w, x[3][e], acc);
+                y[e] = silu_fast(acc);
+            }
         };
         conv(ST_Q, 0, yq);
         conv(ST_K, 1, yk);
@@ -355,7 +365,7 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             unpack8(*(const uint4 *)(stg + ST_G + toff), x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float gv = fmaxf(-gscale * softplusf_(x[e] + DTB[c0 + e]), p.g_lb);
+                const float gv = fmaxf(-gscale * softplus_fast(x[e] + DTB[c0 + e]), p.g_lb);
                 Gh[e] = ti < nvalid ? gv : 0.0f;
             }
         }
@@ -410,16 +420,20 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto qk_at = [&](const uint8_t *stg, const uint8_t *prv, bool first, int t, int c, bool is_q) -> float {
         const int st_off = is_q ? ST_Q : ST_K;
         const int tensor = is_q ? 0 : 1;
-        float acc = 0.0f;
+        float x[4];
         for (int u = 0; u < 4; ++u) {
             const int r = t - 3 + u;
-            float x = 0.0f;
             const int cc = c & 63, off_c = (c >> 6) * CBT + 2 * (cc & 7);
-            if (r >= 0) x = __bfloat162float(*(const __nv_bfloat16 *)(stg + st_off + off_c + swz(r, cc >> 3)));
-            else if (!first) x = __bfloat162float(*(const __nv_bfloat16 *)(prv + st_off + off_c + swz(r + CK, cc >> 3)));
-            acc += CW[(tensor * DD + c) * 4 + u] * x;
+            x[u] = 0.0f;
+            if (r >= 0) x[u] = __bfloat162float(*(const __nv_bfloat16 *)(stg + st_off + off_c + swz(r, cc >> 3)));
+            else if (!first) x[u] = __bfloat162float(*(const __nv_bfloat16 *)(prv + st_off + off_c + swz(r + CK, cc >> 3)));
         }
-        const float y = siluf_(acc);
+        const float4 w = *(const float4 *)(CW + (tensor * DD + c) * 4);
+        float acc = w.x * x[0];
+        acc = fmaf(w.y, x[1], acc);
+        acc = fmaf(w.z, x[2], acc);
+        acc = fmaf(w.w, x[3], acc);
+        const float y = silu_fast(acc);
         const float *nr = NRM + (is_q ? 0 : 4 * CK);
         return y * rsqrtf(nr[t] + nr[CK + t] + nr[2 * CK + t] + nr[3 * CK + t] + L2_EPS);
     };
@@ -427,7 +441,7 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (t >= nvalid) return 0.0f;
         const int cc = c & 63;
         const float x = __bfloat162float(*(const __nv_bfloat16 *)(stg + ST_G + (c >> 6) * CBT + swz(t, cc >> 3) + 2 * (cc & 7)));
-        return fmaxf(-gscale * softplusf_(x + DTB[c]), p.g_lb);
+        return fmaxf(-gscale * softplus_fast(x + DTB[c]), p.g_lb);
     };
 
     bool alive = nchunks > 0 && prep_ab(0);
@@ -551,7 +565,7 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mma_wait();
         tc_fence_after();
 
-        // ============================================================ readback -> P (hi, lo), A^T
+        // ============================================================ readback -> P (hi, lo), A
         if (lq < 2) {
             // lane quarter lq = row block: lanes 0..15 its P rows (q side), 16..31 its A rows;
             // column group cg = 8-column chunk m of j.  Block 1's earlier columns sit at D
@@ -597,8 +611,8 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 *(uint4 *)(gr + GR_PH + swz(i, m)) = hi;
                 *(uint4 *)(gr + GR_PL + swz(i, m)) = lo;
             } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) AT[(8 * m + e) * CK + i] = vals[e];
+                *(float4 *)(A32 + i * AST + 8 * m) = make_float4(vals[0], vals[1], vals[2], vals[3]);
+                *(float4 *)(A32 + i * AST + 8 * m + 4) = make_float4(vals[4], vals[5], vals[6], vals[7]);
             }
         }
         __syncthreads();
@@ -611,39 +625,40 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             issue_tma(n + 1);
         }
 
-        // ============================================================ T (warps 0..7) || Y, O init (warps 8..15)
-        if (warp < 8) {
-            // T = (I + A)^{-1} Diag(beta) by forward substitution, column-parallel: warp w owns
-            // columns w, 15 - w, 16 + w, 31 - w of L^{-1} = (I + A)^{-1}, lane l row l; step m
-            // broadcasts x_m of each column and updates the rows below it (a step before a
-            // column's index leaves it unchanged: its x_m is zero).  All fp32.
-            int colv[4];
+        // ============================================================ T (warp 0) || Y, O init (warps 8..15)
+        if (warp == 0) {
+            // T = (I + A)^{-1} Diag(beta): lane j solves column j of L = I + A in its registers,
+            // left-looking: x_i = -sum_{m < i} A[i][m] x_m for i > j, x_j = 1.  Every lane reads
+            // the same row segment of A (a broadcast); the loops unroll completely.  All fp32.
+            const int j = lane;
+            float x[CK];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) colv[q] = 16 * (q >> 1) + ((q & 1) ? 15 - warp : warp);
-            float x[4];
+            for (int i = 0; i < CK; ++i) x[i] = i == j ? 1.0f : 0.0f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) x[q] = lane == colv[q] ? 1.0f : 0.0f;
-#pragma unroll 4
-            for (int m = 0; m < CK - 1; ++m) {
-                const float am = AT[m * CK + lane];
+            for (int i = 1; i < CK; ++i) {
+                float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float xm = __shfl_sync(0xffffffffu, x[q], m);
-                    x[q] = lane > m ? x[q] - am * xm : x[q];
+                for (int m4 = 0; m4 < i; m4 += 4) {
+                    const float4 av = *(const float4 *)(A32 + i * AST + m4);
+                    acc0 = fmaf(av.x, x[m4], acc0);
+                    if (m4 + 1 < i) acc1 = fmaf(av.y, x[m4 + 1], acc1);
+                    if (m4 + 2 < i) acc0 = fmaf(av.z, x[m4 + 2], acc0);
+                    if (m4 + 3 < i) acc1 = fmaf(av.w, x[m4 + 3], acc1);
                 }
+                x[i] = i == j ? 1.0f : -(acc0 + acc1);
             }
             // T hi, lo in bf16, K-major [i][j]; above the diagonal x is zero
+            const float bj = BETAsm[j];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int j = colv[q];
-                const float tv = x[q] * BETAsm[j];
+            for (int i = 0; i < CK; ++i) {
+                const float tv = x[i] * bj;
                 const __nv_bfloat16 th_ = __float2bfloat16_rn(tv);
-                const uint32_t o = swz(lane, j >> 3) + 2 * (j & 7);
+                const uint32_t o = swz(i, j >> 3) + 2 * (j & 7);
                 *(__nv_bfloat16 *)(gr + GR_TH + o) = th_;
                 *(__nv_bfloat16 *)(gr + GR_TL + o) = __float2bfloat16_rn(tv - __bfloat162float(th_));
             }
             fence_proxy_async();
-        } else {
+        } else if (warp >= 8) {
             const int hb = (warp - 8) >> 2;   // column half of the state this warp splits
             // S^T (fp32, key channels 64 hb ..) -> bf16 hi + lo for the Y and O-init MMAs, which
             // read only these copies, so the state is decayed by exp(G_C) in the same pass
@@ -780,12 +795,31 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 o[e] = __uint_as_float(r[e]);
-                ss[e] = warp_sum(o[e] * o[e]);
+                ss[e] = o[e] * o[e];
             }
-            if (lane == 0) {
+            // sums over the warp's 32 value columns of the 8 tokens by a reduce-scatter: after
+            // the xor-16, -8 and -4 steps lane l holds token (l >> 2) & 7's partial over 8 lanes,
+            // the xor-2 and -1 steps complete it
 #pragma unroll
-                for (int e = 0; e < 8; ++e) RMS[lq * CK + 8 * cg + e] = ss[e];
+            for (int k = 0; k < 4; ++k) {
+                const bool up = lane & 16;
+                const float send = up ? ss[k] : ss[4 + k];
+                ss[k] = (up ? ss[4 + k] : ss[k]) + __shfl_xor_sync(0xffffffffu, send, 16);
             }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const bool up = lane & 8;
+                const float send = up ? ss[k] : ss[2 + k];
+                ss[k] = (up ? ss[2 + k] : ss[k]) + __shfl_xor_sync(0xffffffffu, send, 8);
+            }
+            {
+                const bool up = lane & 4;
+                const float send = up ? ss[0] : ss[1];
+                ss[0] = (up ? ss[1] : ss[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+            }
+            ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 2);
+            ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 1);
+            if ((lane & 3) == 0) RMS[lq * CK + 8 * cg + ((lane >> 2) & 7)] = ss[0];
             __syncthreads();
             const float gain = GAIN[v];
             const uint32_t vo = (v >> 6) * CBT + 2 * (v & 7);
@@ -797,7 +831,7 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float y = __bfloat162float(__float2bfloat16_rn(o[e] * rr)) * gain;   // cast to bf16, then gain
                 const uint32_t eo = vo + swz(i, (v & 63) >> 3);
                 const float zv = __bfloat162float(*(const __nv_bfloat16 *)(stg + ST_Z + eo));
-                *(__nv_bfloat16 *)(stg + ST_G + eo) = __float2bfloat16_rn(y * sigmoidf_(zv));
+                *(__nv_bfloat16 *)(stg + ST_G + eo) = __float2bfloat16_rn(y * sigmoid_fast(zv));
             }
         }
         fence_proxy_async();
