@@ -62,17 +62,20 @@ constexpr int OFF_STG0 = 0, OFF_STG1 = STAGE;
 // Gram region: rows R = [Q_0; K_0; Q_1; K_1] (64 rows x 128 channels, hi and lo, K-major), the
 // M = 128 MMA also reads the 64 rows after each channel block (other operands; the tensor-memory
 // lanes they produce are never read); columns CV (48 rows: tokens 0..31 with their own block's
-// reference, then block 0's tokens with block 1's), hi and lo.  After the Gram: P hi, lo and T
+// reference, then block 0's tokens with block 1's), hi then lo in one 96-row block per channel
+// block, so that R_hi [CV_hi; CV_lo] is one N = 96 MMA.  After the Gram: P hi, lo and T
 // hi, lo ([32 rows][128 B], K-major, columns 0..31 used) and A (fp32 [32][AST], row-major).
 constexpr int OFF_GR = 2 * STAGE;
-constexpr int R_CB = 8192, CV_CB = 6144;
-constexpr int GR_RH = 0, GR_RL = 16384, GR_CVH = 32768, GR_CVL = 32768 + 2 * CV_CB;
-constexpr int GR_BYTES = GR_CVL + 2 * CV_CB;
+constexpr int R_CB = 8192, CV_CB = 12288, CV_LO = 6144;   // CV_lo rows follow CV_hi in a block
+constexpr int GR_RH = 0, GR_RL = 16384, GR_CV = 32768;
+constexpr int GR_BYTES = GR_CV + 2 * CV_CB;
 constexpr int GR_PH = 0, GR_PL = 4096, GR_TH = 8192, GR_TL = 12288, GR_A = 16384, AST = 36;
 // operand tiles ([32 rows][128 channels] bf16, the tile layout)
-constexpr int OFF_QH = OFF_GR + GR_BYTES, OFF_QL = OFF_QH + TILE;   // Q^ hi, lo (K-major B of the O init)
-constexpr int OFF_KH = OFF_QL + TILE;                               // K^ (K-major B of Y)
-constexpr int OFF_KTH = OFF_KH + TILE, OFF_KTL = OFF_KTH + TILE;    // K~ hi, lo (MN-major B of the state update)
+// [Q^_hi; K^] per channel block (32 + 32 rows): one N = 64 B operand gives O and Y into adjacent
+// tensor-memory columns; then Q^ lo (the tile layout)
+constexpr int OFF_QK = OFF_GR + GR_BYTES, QK_CB = 8192, QK_K = 4096;
+constexpr int OFF_QL = OFF_QK + 2 * QK_CB;
+constexpr int OFF_KTH = OFF_QL + TILE, OFF_KTL = OFF_KTH + TILE;    // K~ hi, lo (MN-major B of the state update)
 constexpr int OFF_VH = OFF_KTL + TILE, OFF_VL = OFF_VH + TILE;      // V hi, lo (MN-major A of U)
 constexpr int OFF_CW = OFF_VL + TILE;                               // conv weights fp32 [3][128][4]
 // per-(block, channel) table, fp32 rows of FSTRIDE: fG, fL, fM for blocks 0, 1; the half-block
@@ -95,18 +98,18 @@ constexpr int MS_TSLOT = 4064, MS_ABORT = 4068;
 constexpr int MISC_BYTES = 4096;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-static_assert(OFF_GR % 1024 == 0 && OFF_QH % 1024 == 0 && OFF_VL % 1024 == 0 && GR_CVL % 1024 == 0 &&
-              (GR_CVH + CV_CB) % 1024 == 0, "operand tiles are 1024-aligned");
+static_assert(OFF_GR % 1024 == 0 && OFF_QK % 1024 == 0 && OFF_VL % 1024 == 0 && GR_CV % 1024 == 0 &&
+              CV_LO % 1024 == 0, "operand tiles are 1024-aligned");
 static_assert(GR_A + 32 * AST * 4 <= GR_BYTES && OFF_MISC % 16 == 0, "layout");
 
 // tensor memory columns
 constexpr uint32_t TM_S = 0;     // fp32 S^T, 128
 constexpr uint32_t TM_SH = 128;  // bf16 S^T hi (two per column), 64
 constexpr uint32_t TM_SL = 192;  // bf16 S^T lo, 64
-constexpr uint32_t TM_G = 256;   // Gram D (lanes 0..63), 48
-constexpr uint32_t TM_O = 304;   // O^T, 32
-constexpr uint32_t TM_U = 336;   // U^T, 32
-constexpr uint32_t TM_Y = 368;   // Y^T, 32
+constexpr uint32_t TM_G = 256;   // Gram D (lanes 0..63): R CV_hi in 48 columns, R_hi CV_lo in the next 48
+constexpr uint32_t TM_O = 304;   // O^T, 32 (after the Gram readback)
+constexpr uint32_t TM_Y = 336;   // Y^T, 32 (right after O: one N = 64 accumulator)
+constexpr uint32_t TM_U = 368;   // U^T, 32
 constexpr uint32_t TM_HI = 400;  // bf16 Y^T hi, then U^T hi, 16
 constexpr uint32_t TM_LO = 416;  // bf16 Y^T lo, then U^T lo, 16
 
@@ -260,6 +263,9 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     };
 
     constexpr uint32_t id_gram = idesc_bf16(128, 48, false, false);
+    constexpr uint32_t id_gram96 = idesc_bf16(128, 96, false, false);
+    constexpr uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+    static_assert(TM_Y == TM_O + 32 && TM_G + 96 <= TM_HI, "accumulator layout");
     constexpr uint32_t id_n32 = idesc_bf16(128, 32, false, false);
     constexpr uint32_t id_n32_neg = idesc_bf16(128, 32, false, false, true);
     constexpr uint32_t id_v = idesc_bf16(128, 32, true, false);
@@ -491,11 +497,11 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 o[e] = qf[e] * gam[e];
             }
             split8(o, hi, lo);
-            *(uint4 *)(sm + OFF_QH + toff) = hi;
+            *(uint4 *)(sm + OFF_QK + cb * QK_CB + swz(ti, ca)) = hi;
             *(uint4 *)(sm + OFF_QL + toff) = lo;
 #pragma unroll
             for (int e = 0; e < 8; ++e) o[e] = kf[e] * gam[e];
-            *(uint4 *)(sm + OFF_KH + toff) = pack8(o);
+            *(uint4 *)(sm + OFF_QK + cb * QK_CB + QK_K + swz(ti, ca)) = pack8(o);
             // K~ = exp(G_C - G_i) k = k (E2 / SC) fL
             ftab(FT_L + Bk, f);
 #pragma unroll
@@ -532,16 +538,16 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
             for (int e = 0; e < 8; ++e) o[e] = (badbits >> e & 1u) ? 0.0f : kf[e] * (E2[e] * f[e]);
             split8(o, hi, lo);
-            *(uint4 *)(gr + GR_CVH + cb * CV_CB + swz(ti, ca)) = hi;
-            *(uint4 *)(gr + GR_CVL + cb * CV_CB + swz(ti, ca)) = lo;
+            *(uint4 *)(gr + GR_CV + cb * CV_CB + swz(ti, ca)) = hi;
+            *(uint4 *)(gr + GR_CV + cb * CV_CB + CV_LO + swz(ti, ca)) = lo;
             // Gram columns of block 0's tokens for block 1's rows: k (E2 / SC) fC
             if (Bk == 0) {
                 ftab(FT_C, f);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = kf[e] * ((E2[e] * INV_SC) * f[e]);
                 split8(o, hi, lo);
-                *(uint4 *)(gr + GR_CVH + cb * CV_CB + swz(CK + ti, ca)) = hi;
-                *(uint4 *)(gr + GR_CVL + cb * CV_CB + swz(CK + ti, ca)) = lo;
+                *(uint4 *)(gr + GR_CV + cb * CV_CB + swz(CK + ti, ca)) = hi;
+                *(uint4 *)(gr + GR_CV + cb * CV_CB + CV_LO + swz(CK + ti, ca)) = lo;
             }
         }
         fence_proxy_async();
@@ -549,16 +555,14 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncthreads();
         if (*abort_flag) break;   // the previous chunk's state wait gave up
 
-        // ============================================================ Gram: R_hi CV_hi + R_lo CV_hi + R_hi CV_lo
+        // ============================================================ Gram: R_hi [CV_hi; CV_lo] (N = 96) + R_lo CV_hi
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t sRH = smem_u32(gr + GR_RH), sRL = smem_u32(gr + GR_RL);
-            const uint32_t sCH = smem_u32(gr + GR_CVH), sCL = smem_u32(gr + GR_CVL);
+            const uint32_t sRH = smem_u32(gr + GR_RH), sRL = smem_u32(gr + GR_RL), sCV = smem_u32(gr + GR_CV);
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t orr = (kk >> 2) * R_CB + (kk & 3) * 32, oc = (kk >> 2) * CV_CB + (kk & 3) * 32;
-                mma_ss(tmem + TM_G, sdesc(sRH + orr, 16, 1024), sdesc(sCH + oc, 16, 1024), id_gram, kk > 0);
-                mma_ss(tmem + TM_G, sdesc(sRL + orr, 16, 1024), sdesc(sCH + oc, 16, 1024), id_gram, 1);
-                mma_ss(tmem + TM_G, sdesc(sRH + orr, 16, 1024), sdesc(sCL + oc, 16, 1024), id_gram, 1);
+                mma_ss(tmem + TM_G, sdesc(sRH + orr, 16, 1024), sdesc(sCV + oc, 16, 1024), id_gram96, kk > 0);
+                mma_ss(tmem + TM_G, sdesc(sRL + orr, 16, 1024), sdesc(sCV + oc, 16, 1024), id_gram, 1);
             }
             mma_commit(bar_mma);
         }
@@ -576,16 +580,17 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float bi = BETAsm[i];
             const float pdiag = (PDsm[i] + PDsm[CK + i]) + (PDsm[2 * CK + i] + PDsm[3 * CK + i]);
             const int dcol = B == 0 ? (m < 2 ? 8 * m : -1) : (m < 2 ? CK + 8 * m : 8 * m);
-            uint32_t r[8];
+            uint32_t r[8], r2[8];
             if (dcol >= 0) {
                 tmem_ld8(tmem + lane_q + TM_G + dcol, r);
+                tmem_ld8(tmem + lane_q + TM_G + 48 + dcol, r2);   // the R_hi CV_lo term
                 tmem_wait_ld();
             }
             float vals[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int j = 8 * m + e;
-                const float v = dcol >= 0 ? __uint_as_float(r[e]) : 0.0f;
+                const float v = dcol >= 0 ? __uint_as_float(r[e]) + __uint_as_float(r2[e]) : 0.0f;
                 vals[e] = is_q ? (j < i ? v : (j == i ? pdiag : 0.0f)) : (j < i ? bi * v : 0.0f);
             }
             // exact own-block terms of channels below BAD_LOG, recomputed from the raw tiles
@@ -685,21 +690,16 @@ kda_layer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             named_bar_sync(2, 256);
             if (tid == 256) {
-                // Y^T = S_hi^T K^^T + S_lo^T K^^T, then O^T = S_hi Q^_hi + S_lo Q^_hi + S_hi Q^_lo
+                // [O^T | Y^T] = S^T [Q^_hi; K^]^T from S_hi and S_lo (N = 64), then O^T += S_hi Q^_lo
                 tc_fence_after();
-                const uint32_t sK = smem_u32(sm + OFF_KH), sQH = smem_u32(sm + OFF_QH), sQL = smem_u32(sm + OFF_QL);
+                const uint32_t sQK = smem_u32(sm + OFF_QK), sQL = smem_u32(sm + OFF_QL);
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk >> 2) * CBT + (kk & 3) * 32;
-                    mma_ts(tmem + TM_Y, tmem + TM_SH + kk * 8, sdesc(sK + o, 16, 1024), id_n32, kk > 0);
-                    mma_ts(tmem + TM_Y, tmem + TM_SL + kk * 8, sdesc(sK + o, 16, 1024), id_n32, 1);
+                    const uint32_t oqk = (kk >> 2) * QK_CB + (kk & 3) * 32, oql = (kk >> 2) * CBT + (kk & 3) * 32;
+                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQK + oqk, 16, 1024), id_n64, kk > 0);
+                    mma_ts(tmem + TM_O, tmem + TM_SL + kk * 8, sdesc(sQK + oqk, 16, 1024), id_n64, 1);
+                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQL + oql, 16, 1024), id_n32, 1);
                 }
                 mma_commit(bar_y);
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t o = (kk >> 2) * CBT + (kk & 3) * 32;
-                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQH + o, 16, 1024), id_n32, kk > 0);
-                    mma_ts(tmem + TM_O, tmem + TM_SL + kk * 8, sdesc(sQH + o, 16, 1024), id_n32, 1);
-                    mma_ts(tmem + TM_O, tmem + TM_SH + kk * 8, sdesc(sQL + o, 16, 1024), id_n32, 1);
-                }
                 mma_commit(bar_oi);
             }
             if (mbar_wait_bounded(bar_y, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns)) {

@@ -621,6 +621,41 @@ def test_layer_gate_lower_bound(kda, io, d_):
     assert np.max(np.abs(ru - ro)) > 10 * np.max(np.abs(f64(out) - ro))   # the bound matters
 
 
+@pytest.mark.parametrize("graw", [3.0, 1.0])
+def test_layer_extreme_gates(kda, graw):
+    """The layer kernel's exact diagonal path: with exp(A_log) = 8 and g_raw = 3 every token
+    decays each channel by about e^-24, so every 16-token block is far below the e^-168 the
+    midpoint factorisation takes (the kernel recomputes q, k and g of those channels from the
+    raw tiles); g_raw = 1.0 puts about half the blocks on each side of it.  Against the oracle."""
+    d = inputs.layer_inputs(2, 150, 3, 128, 128, io="bf16", seed=77, s0_std=0.05, dt_bias_std=0.2)
+    d["A_log"] = torch.full_like(d["A_log"], float(np.log(8.0)))
+    d["g_raw"] = (torch.full_like(d["g_raw"], graw).float() +
+                  0.3 * torch.randn(d["g_raw"].shape, generator=torch.Generator().manual_seed(78))).to(torch.bfloat16)
+    out, sT = run_layer(kda, d)
+    ro, rs = oracle_layer(d, torch.bfloat16)
+    assert err(f64(out), ro, torch.bfloat16, stored_bf16=2) <= 1.0
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
+def test_layer_a_wait_that_runs_out_reports_timeout(kda):
+    """The fused layer kernel shares the bounded waits and the drain of the prefill kernel: a
+    tile load that is never issued (chunk 2 of 5) makes its wait run out, the call reports
+    KDA_ERR_TIMEOUT once, and the next call matches the oracle."""
+    d = inputs.layer_inputs(2, 150, 3, 128, 128, io="bf16", seed=79, s0_std=0.05)
+    kda.kda_set_wait_test_hooks(1_000_000, 2)
+    try:
+        with pytest.raises(kda.KdaError) as e:
+            run_layer(kda, d)
+        assert e.value.status == 5
+    finally:
+        kda.kda_set_wait_test_hooks(0, -1)
+    kda.kda_check_device_error()
+    out, sT = run_layer(kda, d)
+    ro, rs = oracle_layer(d, torch.bfloat16)
+    assert err(f64(out), ro, torch.bfloat16, stored_bf16=2) <= 1.0
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
 def test_layer_workload_B2_T16384_H96_sampled_heads(kda):
     """The full layer workload (bf16, unit gain, zero state) in the benchmark's launch shape."""
     w = inputs.WORKLOADS["layer_bf16_B2_T16384_H96_d128"]
