@@ -139,23 +139,40 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": n}
 
 
-def kernel_source_sha():
+# The source files each profiled kernel is compiled from; a capture stays valid while these
+# are unchanged (a change elsewhere in csrc/ does not void it).
+KERNEL_SOURCES = {
+    "kda_chunk_tc": ("chunk_tc.cu", "tc_common.cuh", "common.cuh", "internal.h"),
+    "kda_chunk_tc_packed": ("chunk_tc.cu", "tc_common.cuh", "common.cuh", "internal.h"),
+    "kda_layer_tc": ("layer_tc.cu", "tc_common.cuh", "common.cuh", "internal.h"),
+    "kda_backward": ("backward.cu", "common.cuh", "internal.h"),
+    "kda_decode": ("decode.cu", "common.cuh", "internal.h"),
+    "kda_layer_decode": ("layer_decode.cu", "common.cuh", "internal.h"),
+}
+
+
+def kernel_source_sha(kernel=None):
+    """16 hex digits of the SHA-256 of `kernel`'s source files (all of csrc/ if None or unknown)."""
     import glob
+    csrc = os.path.join(ROOT, "gated_delta_rule_155_b200", "csrc")
+    names = KERNEL_SOURCES.get(kernel)
+    paths = ([os.path.join(csrc, f) for f in names] if names
+             else sorted(glob.glob(os.path.join(csrc, "*"))))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_155_b200", "csrc", "*"))):
+    for p in paths:
         h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
 def traffic_for(kernel):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the kernel sources
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if the kernel's sources
     have not changed since it was captured; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -471,6 +488,7 @@ def run_ours(args):
             "ms_per_step": round(ms_l, 3), "workspace_bytes": need,
             "roofline": {"bound": "hbm", "achieved": round(gbs_l, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs_l / pk["hbm_gbs"], 4),
+                         "traffic": traffic_for("kda_layer_tc") if need == 0 else None,
                          "bytes_per_step": bytes_l}}
         launches_per["layer"] = (3 if need else 1) * nl
         del Ld, ol, sl, wsp, L

@@ -61,10 +61,20 @@ def test_traffic_lookup_requires_the_captured_sources(monkeypatch, tmp_path):
         "k_same": {"source_sha": sha, "dram_bytes_per_launch": 123},
         "k_old": {"source_sha": "0" * 16, "dram_bytes_per_launch": 456}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_sha", lambda: sha)
+    monkeypatch.setattr(bench, "kernel_source_sha", lambda kernel=None: sha)
     assert bench.traffic_for("k_same") == 123
     assert bench.traffic_for("k_old") is None        # kernel changed since the capture
     assert bench.traffic_for("missing") is None
+
+
+def test_each_profiled_kernel_hashes_its_own_sources():
+    bench = _bench_module()
+    for k, files in bench.KERNEL_SOURCES.items():
+        for f in files:
+            assert os.path.exists(os.path.join(ROOT, "gated_delta_rule_155_b200", "csrc", f)), (k, f)
+    # the prefill and the backward are compiled from different files, so their hashes differ
+    assert bench.kernel_source_sha("kda_chunk_tc") != bench.kernel_source_sha("kda_backward")
+    assert bench.kernel_source_sha("kda_chunk_tc") == bench.kernel_source_sha("kda_chunk_tc_packed")
 
 
 def test_reference_arm_prints_one_json_line():
