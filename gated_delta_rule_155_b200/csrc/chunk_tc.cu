@@ -104,7 +104,8 @@ constexpr int MS_TSLOT = 1896;                   // uint32
 constexpr int MS_ABORT = 1900;                   // int
 constexpr int MS_DRAIN = 1904;                   // uint64: MMA drain after an abort
 constexpr int MS_BRAW = 1920;                    // uint32 [2][64]: beta words in flight (cp.async)
-constexpr int MISC_BYTES = 2432;
+constexpr int MS_BAROC = 2432;                   // uint64: the chunk's O MMAs
+constexpr int MISC_BYTES = 2448;
 constexpr int SMEM_BYTES = OFF_MISC + MISC_BYTES + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 static_assert(OFF_LINV + 64 * AST * 4 <= OFF_MISC, "L^{-1} stays clear of the barriers");
@@ -176,6 +177,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint32_t *tslot = (uint32_t *)(misc + MS_TSLOT);
     volatile int *abort_flag = (volatile int *)(misc + MS_ABORT);
     uint64_t *bar_drain = (uint64_t *)(misc + MS_DRAIN);
+    uint64_t *bar_oc = (uint64_t *)(misc + MS_BAROC);
     float *A32 = (float *)(sm + OFF_A32);
     float *LINV = (float *)(sm + OFF_LINV);
 
@@ -198,6 +200,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(bar_mma, 1);
         mbar_init(bar_o, 1);
         mbar_init(bar_y, 1);
+        mbar_init(bar_oc, 1);
         mbar_init(bar_drain, 3);   // the three MMA-issuing threads
         *abort_flag = 0;
         for (int i = 0; i < 16; ++i) badmask[i] = 0u;
@@ -389,8 +392,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (Bq == 0) GCsm[c] = __expf(Lv[0] + Lv[1] + Lv[2] + Lv[3]);
         }
         // the previous chunk's O tile (its stage region takes this chunk's Gram operands in pass
-        // C) must have been read out by its TMA store
+        // C) must have been read out by its TMA store, and its state-update MMAs, which read K~
+        // hi and lo where pass C writes the Gram operands, must have completed (they ran under
+        // the O staging, the store and passes A and B)
         if (tid == 0) bulk_wait_read_all();
+        if (n > 0) mma_wait();
         __syncthreads();
         // pass C, per token.  With SC = 2^120:
         //   E1 = SC exp(G_i - G_blockstart)  (includes token i)
@@ -527,6 +533,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
+        if (*abort_flag) break;   // the previous chunk's state-update wait gave up
 
         // ============================================================ Gram (MMA)
         if (tid == 0) {
@@ -889,6 +896,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_ts(tmem + TM_O, tmem + TM_LO32 + kk * 8, sdesc(sP + kk * 32, 16, 1024), id_op, 1);
                 mma_ts(tmem + TM_O, tmem + TM_HI32 + kk * 8, sdesc(sPL + kk * 32, 16, 1024), id_op, 1);
             }
+            mma_commit(bar_oc);   // O is read out while the state update runs
             for (int kk = 0; kk < 4; ++kk) {
                 mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
                 mma_ts(tmem + TM_S, tmem + TM_LO32 + kk * 8, sdesc(sG + kk * 2048, 8192, 1024), id_s, 1);
@@ -896,9 +904,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mma_ts(tmem + TM_S, tmem + TM_HI32 + kk * 8, sdesc(sKL0 + kk * 2048, 8192, 1024), id_s64, 1);
                 mma_ts(tmem + TM_S + 64, tmem + TM_HI32 + kk * 8, sdesc(sKL1 + kk * 2048, 8192, 1024), id_s64, 1);
             }
-            mma_commit(bar_mma);
+            mma_commit(bar_mma);   // waited for before the next chunk's pass C (or the final state)
         }
-        mma_wait();
+        mbar_wait_bounded(bar_oc, (uint32_t)(n & 1), abort_flag, p.err, p.wait_ns);
         tc_fence_after();
         {
             // O^T -> bf16 tile in the stage's V tile (dead since the U~ MMA; the load tiles'
@@ -917,7 +925,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (*abort_flag) break;   // the O / state wait gave up
+        if (*abort_flag) break;   // the O wait gave up
         if (tail) {
             // the last chunk of a packed sequence: its tile's later rows are the next
             // sequence's, so only the valid rows are written, 16 bytes per thread and pass
@@ -935,6 +943,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
 
     // ---------------------------------------------------------------- final state
+    // The flag has not changed since its last check after a block barrier, so every thread
+    // takes the same branch; the last chunk's state update is still running.
+    if (nchunks > 0 && !*abort_flag) {
+        mma_wait();
+        tc_fence_after();
+    }
+    __syncthreads();
     if (p.sT && !*abort_flag) {
         tc_fence_after();
         const int v = 32 * lq + lane;
