@@ -22,9 +22,9 @@
 //   dg = reverse cumsum of dG;   dS = Diag(exp G_C) dS_next + Q^^T dO - K^^T dX.
 // Every exponent is a sum of non-positive log-decays, so nothing overflows for any gate.
 //
-// One CTA of 512 threads per (b, h).  A forward sweep writes the chunk-start states to the
-// workspace (checkpoints); the reverse sweep reloads each one, recomputes the chunk's
-// forward quantities and applies the lines above, with dS held in shared memory.
+// One CTA of 512 threads per (b, h).  A forward sweep writes, per chunk, the chunk-start state
+// and the chunk's forward quantities (Abar, P, M, X, U) to the workspace; the reverse sweep
+// reloads them and applies the lines above, with dS held in shared memory.
 #include "common.cuh"
 #include "internal.h"
 
@@ -63,8 +63,16 @@ struct BwdArgs {
     const float *dST;                   // [B, H, D, D] or null
     void *dq, *dk, *dv, *dg, *dbeta;    // io dtype
     float *ds0;                         // [B, H, D, D] or null
-    float *ckpt;                        // [B, H, nchunks, D, D]
+    float *ckpt;                        // [B, H, nchunks, ChunkRecord<D>::FLOATS]
     int T, H;
+};
+
+// What the forward sweep keeps of each chunk (fp32): the chunk-start state [D][D], U and X =
+// V - K^ S [BC][D], then M, P and Abar [BC][BC] (dense).
+template <int D>
+struct ChunkRecord {
+    static constexpr int S = 0, U = D * D, X = U + BC * D, M = X + BC * D, P = M + BC * BC, AB = P + BC * BC;
+    static constexpr int FLOATS = AB + BC * BC;
 };
 
 template <typename IO, int D>
@@ -85,7 +93,8 @@ kda_backward_kernel(BwdArgs a)
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int T = a.T, H = a.H;
     const int nch = (T + BC - 1) / BC;
-    float *ck = a.ckpt + (size_t)bh * nch * D * D;
+    using R = ChunkRecord<D>;
+    float *ck = a.ckpt + (size_t)bh * nch * R::FLOATS;
     const size_t soff = (size_t)bh * D * D;
     const int col = tid % D, rb = tid / D;   // column and row block (or value block) of this thread
     auto gidx = [&](int t, int c) -> size_t { return ((size_t)(b * T + t) * H + h) * D + c; };
@@ -255,22 +264,35 @@ kda_backward_kernel(BwdArgs a)
     __syncthreads();
     for (int n = 0; n < nch; ++n) {
         const int t0 = n * BC;
-        store_state(ck + (size_t)n * D * D, Ss);
+        float *rec = ck + (size_t)n * R::FLOATS;
+        store_state(rec + R::S, Ss);
         {
-            float *const dst[3] = {Ks, Gs, Vs};
-            const void *const src[3] = {a.k, a.g, a.v};
-            load_chunk(dst, src, 3, t0, nullptr, nullptr);
+            float *const dst[4] = {Qs, Ks, Gs, Vs};
+            const void *const src[4] = {a.q, a.k, a.g, a.v};
+            load_chunk(dst, src, 4, t0, nullptr, nullptr);
         }
         if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         gates(false);
-        pair_dots(false);
+        pair_dots(true);
         __syncthreads();
         if (warp == 0) invert();
         ks_x();
         __syncthreads();
         u_from_x();
         __syncthreads();
+        // the chunk's record for the reverse sweep: U, X (in Vs), M, P, Abar
+        for (int idx = tid; idx < BC * D / 4; idx += BNT) {
+            const int i = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+            *(float4 *)(rec + R::U + i * D + c4) = *(const float4 *)(Us + i * LD + c4);
+            *(float4 *)(rec + R::X + i * D + c4) = *(const float4 *)(Vs + i * LD + c4);
+        }
+        if (tid < BC * BC) {
+            const int i = tid / BC, j = tid % BC;
+            rec[R::M + tid] = Ms[i * CL + j];
+            rec[R::P + tid] = j <= i ? Ps[i * CL + j] : 0.0f;
+            rec[R::AB + tid] = j < i ? ABs[i * CL + j] : 0.0f;
+        }
         // S <- Diag(exp G_C) S + K~^T U; (column, value block) partition
         {
             const float gc = __expf(GCs[col]);
@@ -299,20 +321,47 @@ kda_backward_kernel(BwdArgs a)
     load_state(dSs, a.dST ? a.dST + soff : nullptr);
     for (int n = nch - 1; n >= 0; --n) {
         const int t0 = n * BC;
+        const float *rec = ck + (size_t)n * R::FLOATS;
         {
-            float *const dst[5] = {Qs, Ks, Gs, Vs, dOs};
-            const void *const src[5] = {a.q, a.k, a.g, a.v, a.dO};
-            load_chunk(dst, src, 5, t0, Ss, ck + (size_t)n * D * D);
+            // the record's U, X, M, P, Abar: loads issued before the chunk's, stored after
+            constexpr int NF4 = BC * D / 4, UX = (NF4 + BNT - 1) / BNT;   // float4s of U (of X) per thread
+            static_assert(BC * BC <= BNT, "record load mapping");
+            float4 ru[UX], rx[UX];
+#pragma unroll
+            for (int e = 0; e < UX; ++e) {
+                const int idx = tid + BNT * e, i = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+                if (idx < NF4) {
+                    ru[e] = *(const float4 *)(rec + R::U + i * D + c4);
+                    rx[e] = *(const float4 *)(rec + R::X + i * D + c4);
+                }
+            }
+            float rm = 0.0f, rp = 0.0f, ra = 0.0f;
+            if (tid < BC * BC) {
+                rm = rec[R::M + tid];
+                rp = rec[R::P + tid];
+                ra = rec[R::AB + tid];
+            }
+            float *const dst[4] = {Qs, Ks, Gs, dOs};
+            const void *const src[4] = {a.q, a.k, a.g, a.dO};
+            load_chunk(dst, src, 4, t0, Ss, rec + R::S);
+#pragma unroll
+            for (int e = 0; e < UX; ++e) {
+                const int idx = tid + BNT * e, i = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+                if (idx < NF4) {
+                    *(float4 *)(Us + i * LD + c4) = ru[e];
+                    *(float4 *)(Vs + i * LD + c4) = rx[e];   // X
+                }
+            }
+            if (tid < BC * BC) {
+                const int i = tid / BC, j = tid % BC;
+                Ms[i * CL + j] = rm;
+                Ps[i * CL + j] = rp;
+                ABs[i * CL + j] = ra;
+            }
         }
         if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         gates(true);
-        pair_dots(true);
-        __syncthreads();
-        if (warp == 0) invert();
-        ks_x();
-        __syncthreads();
-        u_from_x();
         __syncthreads();
 
         // dU = P^T dO + K~ dS_next, (row block, column) partition; then per (row, channel):
@@ -528,7 +577,8 @@ cudaError_t launch_bwd_t(const BwdArgs &a, int B, cudaStream_t s)
 size_t backward_workspace_bytes(int B, int T, int H, int d)
 {
     const size_t nch = (size_t)(T + BC - 1) / BC;
-    return (size_t)B * H * nch * d * d * sizeof(float);
+    const size_t rec = d == 128 ? ChunkRecord<128>::FLOATS : ChunkRecord<64>::FLOATS;
+    return (size_t)B * H * nch * rec * sizeof(float);
 }
 
 cudaError_t launch_backward(const BackwardArgs &x, cudaStream_t s)

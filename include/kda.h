@@ -96,8 +96,10 @@ kda_status_t kda_forward_chunked(const void *q, const void *k, const void *v, co
                                  int chunk, kda_dtype_t io, kda_stream_t stream);
 
 /*
- * Bytes of device workspace kda_backward_chunked needs: the fp32 state at the start of
- * every 16-token chunk, B * H * ceil(T / 16) * dk * dv * 4.  dk must equal dv
+ * Bytes of device workspace kda_backward_chunked needs: for every 16-token chunk, the fp32
+ * state at its start (d * d floats) and the chunk's forward quantities U and X = V - K^ S
+ * (2 * 16 * d floats) and its three 16 x 16 matrices, so
+ * B * H * ceil(T / 16) * (d * d + 32 * d + 768) * 4 with d = dk.  dk must equal dv
  * (KDA_ERR_UNSUPPORTED otherwise).  *bytes is written on KDA_OK.
  */
 kda_status_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
@@ -107,9 +109,9 @@ kda_status_t kda_backward_workspace_size(int B, int T, int H, int dk, int dv, kd
  * kda_backward_chunked — gradients of the recurrence of kda_forward_chunked (training;
  * the pages' runs differentiate the KDA layer: maxtext PR #5550, its jax.grad test and the
  * C4 training steps).  Given d_out = dL/dout and d_final_state = dL/dS_T, writes dL/d of
- * every input.  Computed in fp32 from the io-dtype inputs: a forward sweep stores the
- * chunk-start states in `workspace`, then a reverse sweep over 16-token chunks recomputes
- * each chunk and applies the chain rule (pairwise decays exp(G_i - G_j), j <= i, so no
+ * every input.  Computed in fp32 from the io-dtype inputs: a forward sweep stores each
+ * 16-token chunk's start state and forward quantities in `workspace`, then a reverse sweep
+ * reloads them and applies the chain rule (pairwise decays exp(G_i - G_j), j <= i, so no
  * gate overflows).
  *   q, k, g, v, beta, initial_state   as kda_forward_chunked (inputs, unchanged)
  *   d_out          [B, T, H, dv] io dtype
@@ -167,8 +169,10 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const 
                              int dv, kda_dtype_t io, kda_stream_t stream);
 
 /*
- * Bytes of device workspace kda_layer_forward needs for these sizes (0 when the
- * selected kernels need none).  *bytes is written on KDA_OK.
+ * Bytes of device workspace kda_layer_forward needs for these sizes.  0 for bf16 at
+ * dk = dv = 128, whose prologue, chunked step and epilogue run as one tensor-core kernel;
+ * otherwise the fp32 prologue outputs and the chunked step's output (q, k, g, v, beta, o in
+ * fp32, each rounded up to 256 bytes).  *bytes is written on KDA_OK.
  */
 kda_status_t kda_layer_workspace_size(int B, int T, int H, int dk, int dv, kda_dtype_t io,
                                       size_t *bytes);

@@ -114,7 +114,8 @@ def test_forward_chunked_varlen_rejects_bad_arguments(lib):
 def test_backward_rejects_bad_arguments(lib):
     n = ctypes.c_size_t(0)
     assert lib.kda_backward_workspace_size(2, 33, 3, 128, 128, 1, ctypes.byref(n)) == 0
-    assert n.value == 2 * 3 * 3 * 128 * 128 * 4          # three 16-token chunks per head
+    # three 16-token chunks per head, each: the state, U and X, and three 16 x 16 matrices
+    assert n.value == 2 * 3 * 3 * (128 * 128 + 2 * 16 * 128 + 3 * 16 * 16) * 4
     assert lib.kda_backward_workspace_size(2, 33, 3, 128, 64, 1, ctypes.byref(n)) == 2
 
     def call(q=A16, ws=A16, ws_bytes=1 << 40, dk=128, dv=128, T=33, dgp=A16):
