@@ -191,27 +191,54 @@ kda_backward_kernel(BwdArgs a)
             if (with_q) QHs[i * LD + c] = Qs[i * LD + c] * e;
         }
     };
-    // Abar (j < i) and, with_p, P (j <= i): one warp per pair, lanes over channels
-    auto pair_dots = [&](bool with_p) {
-        for (int p = warp; p < BC * (BC + 1) / 2; p += BNT / 32) {
-            int i = 0;
-            while ((i + 1) * (i + 2) / 2 <= p) ++i;
-            const int j = p - i * (i + 1) / 2;
-            if (!with_p && j == i) continue;
-            float pv = 0.0f, av = 0.0f;
+    // P (j <= i) and Abar (j < i).  Warp w takes the pairs p = w + 16 k (k < 9) of the 136
+    // (i, j <= i), lanes over channels; the 9 + 9 per-lane partial sums are then reduced in one
+    // transposed butterfly (31 shuffles instead of 18 x 5), after which lane l holds the total
+    // of partial l: P of pair k in lane k, Abar of pair k in lane 16 + k.  The pairing of the
+    // butterfly is warp_sum's, so the sums are the same to the bit.
+    auto pair_dots = [&]() {
+        constexpr int NP = BC * (BC + 1) / 2, KP = (NP + 15) / 16;
+        static_assert(KP <= 16 && BNT / 32 == 16, "pair mapping");
+        float v[32];
 #pragma unroll
-            for (int e = 0; e < D / 32; ++e) {
-                const int c = lane + 32 * e;
-                const float x = Ks[j * LD + c] * __expf(Gs[i * LD + c] - Gs[j * LD + c]);
-                if (with_p) pv += Qs[i * LD + c] * x;
-                av += Ks[i * LD + c] * x;
+        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < KP; ++k) {
+            const int p = warp + 16 * k;
+            if (p < NP) {
+                int i = (int)((sqrtf(8.0f * p + 1.0f) - 1.0f) * 0.5f);
+                if ((i + 1) * (i + 2) / 2 <= p) ++i;
+                if (i * (i + 1) / 2 > p) --i;
+                const int j = p - i * (i + 1) / 2;
+                float pv = 0.0f, av = 0.0f;
+#pragma unroll
+                for (int e = 0; e < D / 32; ++e) {
+                    const int c = lane + 32 * e;
+                    const float x = Ks[j * LD + c] * __expf(Gs[i * LD + c] - Gs[j * LD + c]);
+                    pv += Qs[i * LD + c] * x;
+                    av += Ks[i * LD + c] * x;
+                }
+                v[k] = pv;
+                v[16 + k] = av;
             }
-            pv = warp_sum(pv);
-            av = warp_sum(av);
-            if (lane == 0) {
-                if (with_p) Ps[i * CL + j] = pv;
-                if (j < i) ABs[i * CL + j] = av;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int e = 0; e < o; ++e) {
+                const float keep = up ? v[e + o] : v[e], send = up ? v[e] : v[e + o];
+                v[e] = keep + __shfl_xor_sync(0xffffffffu, send, o);
             }
+        }
+        const int k = lane & 15, p = warp + 16 * k;
+        if (k < KP && p < NP) {
+            int i = (int)((sqrtf(8.0f * p + 1.0f) - 1.0f) * 0.5f);
+            if ((i + 1) * (i + 2) / 2 <= p) ++i;
+            if (i * (i + 1) / 2 > p) --i;
+            const int j = p - i * (i + 1) / 2;
+            if (lane < 16) Ps[i * CL + j] = v[0];
+            else if (j < i) ABs[i * CL + j] = v[0];
         }
     };
     // M = (I + Diag(beta) Abar)^-1 by forward substitution; lane j owns column j (warp 0)
@@ -274,7 +301,7 @@ kda_backward_kernel(BwdArgs a)
         if (tid < BC) BETA[tid] = t0 + tid < T ? to_f32(((const IO *)a.beta)[(size_t)(b * T + t0 + tid) * H + h]) : 0.0f;
         __syncthreads();
         gates(false);
-        pair_dots(true);
+        pair_dots();
         __syncthreads();
         if (warp == 0) invert();
         ks_x();
