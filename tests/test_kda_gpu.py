@@ -544,6 +544,26 @@ def test_backward_workload_B1_T4096_H32_sampled_heads(kda):
         assert serr(f64(gr["d_initial_state"][:, h:h + 1]), ref["ds0"], torch.bfloat16) <= 1.0
 
 
+def test_backward_workload_B4_T8192_H96_sampled_heads(kda):
+    """The backward as the benchmark launches it: the B = 4, T = 8192, H = 96 bf16 prefill
+    workload with dO ~ N(0, 1) (torch generator, seed 7), no state gradients; four heads
+    checked over the whole 8192-token sequence against the reverse-mode oracle."""
+    w = inputs.WORKLOADS["prefill_bf16_B4_T8192_H96_d128"]
+    d = inputs.prefill_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], io=w["io"], seed=w["seed"])
+    gen = torch.Generator().manual_seed(7)
+    dO = torch.randn(d["v"].shape, generator=gen).to(torch.bfloat16)
+    gr = run_backward(kda, d, dO, None)
+    for b, h in ((0, 0), (1, 40), (2, 77), (3, 95)):
+        sl = lambda x, b=b, h=h: x[b:b + 1, :, h:h + 1]
+        ref = oracle.recurrent_backward(*(f64(sl(d[n])) for n in ("q", "k", "v", "g", "beta")), None,
+                                        f64(sl(dO)), None, nthreads=1)
+        for name in ("dq", "dk", "dv", "dg", "dbeta"):
+            e = err(f64(sl(gr[name])), ref[name], torch.bfloat16, stored_bf16=True)
+            assert e <= 1.0, f"({b}, {h}) {name}: {e:.3e} of bound"
+        assert serr(f64(gr["d_initial_state"][b:b + 1, h:h + 1]), ref["ds0"], torch.bfloat16) <= 1.0
+    assert all(bool(torch.isfinite(gr[n]).all()) for n in ("dq", "dk", "dv", "dg", "dbeta"))
+
+
 # ------------------------------------------------------------------------ layer
 
 
