@@ -285,17 +285,33 @@ def run_ours(args):
                            "frac": round(flops_launch / (launch_ms / 1e3) / 1e12 / pk["bf16_tflops"], 4)}}
     launches_per["prefill"] = 1
 
-    # e2e through the C ABI from pinned host buffers: H2D inputs, kernel, D2H output
+    # e2e through the C ABI from pinned host buffers: every step copies all inputs host -> device,
+    # runs the prefill and copies the whole output back.  Sequence by sequence on three streams,
+    # so that the copy of sequence b + 1 in, the prefill of sequence b and the copy of sequence
+    # b - 1 out overlap (host->device and device->host use separate copy engines).
     e2e = None
     if "e2e" not in skip:
         out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(B)]
+        ev_done = [torch.cuda.Event() for _ in range(B)]
 
         def e2e_step():
-            with torch.cuda.stream(stream):
-                for n in host:
-                    dv_in[n].copy_(host[n], non_blocking=True)
-                prefill_step()
-                out_host.copy_(out, non_blocking=True)
+            s_in.wait_stream(stream)       # after the step's start event
+            for b in range(B):
+                with torch.cuda.stream(s_in):
+                    for n in host:
+                        dv_in[n][b].copy_(host[n][b], non_blocking=True)
+                    ev_in[b].record(s_in)
+                stream.wait_event(ev_in[b])
+                kda.kda_forward_chunked(dv_in["q"][b:b + 1], dv_in["k"][b:b + 1], dv_in["v"][b:b + 1],
+                                        dv_in["g"][b:b + 1], dv_in["beta"][b:b + 1], None, out[b:b + 1],
+                                        sT[b:b + 1], stream=stream)
+                ev_done[b].record(stream)
+                s_out.wait_event(ev_done[b])
+                with torch.cuda.stream(s_out):
+                    out_host[b].copy_(out[b], non_blocking=True)
+            stream.wait_stream(s_out)      # before the step's end event
 
         ne = max(1, args.e2e_steps)
         tot_e, _ = timed(torch, e2e_step, ne, 1, stream, barrier, per_launch=False)
