@@ -15,7 +15,8 @@
 //   pass C               q, k L2-normalised; Q^ = Gamma q, K^ = Gamma k, K~ = exp(G_C - G) k,
 //                        V, and the Gram operands (the overflow-safe midpoint factorisation of
 //                        the tensor-core prefill, chunk_tc.cu)
-//   Gram (tcgen05)       P (j <= i) and A (j < i) in one M = 128, N = 48, K = 128 MMA group
+//   Gram (tcgen05)       P (j <= i) and A (j < i): R_hi [CV_hi; CV_lo] (M = 128, N = 96) and
+//                        R_lo CV_hi (N = 48), K = 128
 //   inverse || Y, O init T = (I + A)^{-1} Diag(beta), one column per lane in registers, while
 //                        the tensor cores compute Y^T = S^T K^^T and O^T = S^T Q^^T
 //   U, O, S (tcgen05)    U = T (V - Y);  O += P U;  S <- Diag(exp G_C) S + K~^T U
