@@ -423,7 +423,9 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
                          "frac_of_8TBs": round(gbs / 8000.0, 4), "traffic": traffic_for("kda_decode"),
-                         "kernel": "kda_decode", "bytes_per_launch": state_bytes + io_bytes}}
+                         "kernel": "kda_decode", "bytes_per_launch": state_bytes + io_bytes,
+                         "note": "the state is read and written in place (same lines), which a plain "
+                                 "copy's read-A/write-B peak does not model; frac can exceed 1"}}
         launches_per["decode"] = wd["steps"] * reps
         del state, steps_in, od, dd
         torch.cuda.empty_cache()

@@ -6,12 +6,14 @@
 // (the gated delta rule for one token; the fixed-size per-head state is what the
 //  open-model-atlas "Kimi-K3 ?inspect=blocks" page contrasts with the KV cache).
 //
-// The state is read once and written once.  Value columns are independent, so a CTA
-// owns one 64-column slice of one head: 256 threads, 16 threads per row segment of
-// 64 floats (one float4 each, fully coalesced 256-byte row segments), 16 rows per
-// pass, dk/16 passes, issued before anything else.  Each thread keeps its dk/16 decayed
-// float4s in registers between the reduction and the write-back; three CTAs fit per SM.  Column sums over dk reduce first
-// across the two rows a warp holds (shuffle) and then across the 8 warps (smem).
+// The state is read once and written once.  At dk = dv = 128 one CTA of 512 threads owns a
+// head: a warp reads whole 512-byte rows (one float4 per lane), 16 rows per pass, 8 passes,
+// issued before anything else, so 64 KB per CTA are in flight at once; the column sums over dk
+// reduce across the 16 row groups in shared memory.  Other shapes: a CTA owns one 64-column
+// slice of one head, 256 threads, 16 threads per 256-byte row segment, 16 rows per pass; column
+// sums reduce across the two rows a warp holds (shuffle) and then across the 8 warps (smem).
+// Either way each thread keeps its decayed float4s in registers between the reduction and the
+// write-back.
 #include "common.cuh"
 #include "internal.h"
 
@@ -113,9 +115,86 @@ kda_decode_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *
     }
 }
 
+// dk = dv = 128: one CTA of 512 threads per (b, h), whole rows per warp.
+constexpr int DR_THREADS = 512, DR_D = 128, DR_ROWS = DR_THREADS / 32, DR_NPASS = DR_D / DR_ROWS;
+
+template <typename IO>
+__global__ void __launch_bounds__(DR_THREADS, 2)
+kda_decode_row_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
+                      const IO *__restrict__ g, const IO *__restrict__ beta, float *state,
+                      IO *__restrict__ out)
+{
+    __shared__ float s_alpha[DR_D], s_k[DR_D], s_q[DR_D], s_u[DR_D];
+    __shared__ __align__(16) float s_red_a[DR_ROWS][DR_D];
+    __shared__ __align__(16) float s_red_b[DR_ROWS][DR_D];
+    __shared__ float s_qk;
+
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t vec = (size_t)bh * DR_D;
+
+    // the state loads go out first, so their latency overlaps the small vector loads below
+    const int col4 = lane * 4, row0 = warp;
+    float *Sb = state + (size_t)bh * DR_D * DR_D + col4;
+    float4 s[DR_NPASS];
+#pragma unroll
+    for (int p = 0; p < DR_NPASS; ++p) s[p] = *reinterpret_cast<const float4 *>(Sb + (size_t)(row0 + DR_ROWS * p) * DR_D);
+
+    if (tid < DR_D) {
+        s_alpha[tid] = __expf(to_f32(g[vec + tid]));
+        s_k[tid] = to_f32(k[vec + tid]);
+        s_q[tid] = to_f32(q[vec + tid]);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float pq = 0.0f;
+        for (int c = lane; c < DR_D; c += 32) pq += s_q[c] * s_k[c];
+        pq = warp_sum(pq);
+        if (lane == 0) s_qk = pq;
+    }
+    float a4[4] = {0.f, 0.f, 0.f, 0.f}, b4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int p = 0; p < DR_NPASS; ++p) {
+        const int r = row0 + DR_ROWS * p;
+        const float al = s_alpha[r], kr = s_k[r], qr = s_q[r];
+        s[p].x *= al; s[p].y *= al; s[p].z *= al; s[p].w *= al;
+        a4[0] += kr * s[p].x; a4[1] += kr * s[p].y; a4[2] += kr * s[p].z; a4[3] += kr * s[p].w;
+        b4[0] += qr * s[p].x; b4[1] += qr * s[p].y; b4[2] += qr * s[p].z; b4[3] += qr * s[p].w;
+    }
+    *reinterpret_cast<float4 *>(&s_red_a[row0][col4]) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+    *reinterpret_cast<float4 *>(&s_red_b[row0][col4]) = make_float4(b4[0], b4[1], b4[2], b4[3]);
+    __syncthreads();
+    if (tid < DR_D) {
+        float sa = 0.f, sb = 0.f;
+#pragma unroll
+        for (int w = 0; w < DR_ROWS; ++w) {
+            sa += s_red_a[w][tid];
+            sb += s_red_b[w][tid];
+        }
+        const float u = to_f32(beta[bh]) * (to_f32(v[vec + tid]) - sa);
+        s_u[tid] = u;
+        out[vec + tid] = from_f32<IO>(sb + s_qk * u);
+    }
+    __syncthreads();
+    const float u0 = s_u[col4], u1 = s_u[col4 + 1], u2 = s_u[col4 + 2], u3 = s_u[col4 + 3];
+#pragma unroll
+    for (int p = 0; p < DR_NPASS; ++p) {
+        const int r = row0 + DR_ROWS * p;
+        const float kr = s_k[r];
+        *reinterpret_cast<float4 *>(Sb + (size_t)r * DR_D) =
+            make_float4(s[p].x + kr * u0, s[p].y + kr * u1, s[p].z + kr * u2, s[p].w + kr * u3);
+    }
+}
+
 template <typename IO, int DK>
 cudaError_t launch_t(const DecodeArgs &a, cudaStream_t s)
 {
+    if (DK == DR_D && a.dv == DR_D) {
+        kda_decode_row_kernel<IO><<<(unsigned)(a.B * a.H), DR_THREADS, 0, s>>>(
+            (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, (const IO *)a.g, (const IO *)a.beta, a.state,
+            (IO *)a.out);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)(a.B * a.H), (unsigned)(a.dv / DEC_SLICE));
     kda_decode_kernel<IO, DK><<<grid, DEC_THREADS, 0, s>>>(
         (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, (const IO *)a.g, (const IO *)a.beta,
