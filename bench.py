@@ -315,6 +315,7 @@ def run_ours(args):
 
         ne = max(1, args.e2e_steps)
         tot_e, _ = timed(torch, e2e_step, ne, 1, stream, barrier, per_launch=False)
+        launches_per["e2e"] = ne * B
         ms_e = max_over_ranks(tot_e / ne)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         e2e = {"value": round(ws * ntok / (ms_e / 1e3), 1), "unit": "tokens/s",
@@ -524,7 +525,7 @@ def run_ours(args):
 
     gpu_launches = args.steps * (launches_per["prefill"] + launches_per.get("varlen", 0)) + \
         launches_per.get("backward", 0) + launches_per.get("decode", 0) + launches_per.get("layer_decode", 0) + \
-        launches_per.get("layer", 0)
+        launches_per.get("layer", 0) + launches_per.get("e2e", 0)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
