@@ -619,6 +619,19 @@ def test_layer_small(kda, io, d_, T):
     assert serr(f64(sT), rs, io) <= 1.0
 
 
+@pytest.mark.parametrize("io,d_", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_layer_zero_length_copies_state(kda, io, d_):
+    """T = 0: no output rows; the final state is the initial state, or zeros without one."""
+    ioname = "f32" if io == torch.float32 else "bf16"
+    d = inputs.layer_inputs(2, 0, 3, d_, d_, io=ioname, seed=47, s0_std=0.1)
+    out, sT = run_layer(kda, d)
+    assert out.numel() == 0
+    assert torch.equal(sT.cpu(), d["s0"])
+    d["s0"] = None
+    _, sT = run_layer(kda, d)
+    assert torch.count_nonzero(sT) == 0
+
+
 def clamped_fraction(d, lb):
     g = oracle.gate(f64(d["g_raw"]), f64(d["A_log"]), None if d["dt_bias"] is None else f64(d["dt_bias"]))
     return float(np.mean(g < lb))
