@@ -740,6 +740,21 @@ def test_layer_varlen_ragged(kda, io, d_):
     assert serr(f64(sT), rs, io) <= 1.0
 
 
+def test_layer_varlen_many_short_sequences(kda):
+    """200 packed sequences of 0..20 tokens (the final states are a few nearly rank-one
+    updates of a small initial state, the case that bounds the state's rounding), bf16 at
+    d = 128 on the fused tensor-core kernel: every output and every final state."""
+    lens = [int(x) for x in np.random.default_rng(93).integers(0, 21, 200)]
+    P = packed_layer_inputs(lens, 2, 128, "bf16", seed=94, s0_std=0.02)
+    out, sT = run_layer_varlen(kda, P)
+    a = {n: (None if v is None else f64(v)) for n, v in P.items()}
+    ro, rs = oracle.layer_varlen(a["q_raw"], a["k_raw"], a["v_raw"], a["conv_q"], a["conv_k"], a["conv_v"],
+                                 a["g_raw"], a["A_log"], a["dt_bias"], a["b_raw"], a["o_gate_raw"],
+                                 P["cu_seqlens"].numpy(), a["o_norm_w"], s0=a["s0"], io_bf16=True)
+    assert err(f64(out), ro, torch.bfloat16, stored_bf16=2) <= tol(torch.bfloat16)
+    assert serr(f64(sT), rs, torch.bfloat16) <= 1.0
+
+
 def test_layer_varlen_equal_lengths_equal_the_batched_layer(kda):
     """Three packed sequences of 70 tokens give kda_layer_forward's B = 3 results bit for bit."""
     P = packed_layer_inputs([70, 70, 70], 2, 128, "bf16", seed=150)
